@@ -1,0 +1,432 @@
+/*
+ * sa3_oracle.c -- plain, slow CPU oracle for microscaled-FP4 attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only tests/, the smoke check in __graft_entry__.py and the
+ * cpu_baseline / reference leg of bench.py use it.  It shares no code, header,
+ * table or helper with the CUDA library; it is written from the method's
+ * definition, step by step, in the order the method states them.
+ *
+ * Sources (pages by title, section):
+ *  - "SageAttention: Accurate 8-Bit Attention for Plug-and-play Inference
+ *    Acceleration" (atlas.scime.ai summary), section "Approach": K is smoothed
+ *    by subtracting its mean over tokens, which leaves softmax attention
+ *    unchanged.                                                   -> kmean()
+ *  - "SageAttention3: Microscaling FP4 Attention for Inference and An
+ *    Exploration of 8-Bit Training" (transistor.fm / mlsanity.com abstract):
+ *    attention computed on Blackwell FP4 tensor cores with microscaled FP4
+ *    operands.                                                    -> quantize
+ *  - references listed on mlsanity.com: "FP8 Formats for Deep Learning"
+ *    (E4M3 scale format) and "Microscaling Data Formats for Deep Learning"
+ *    (E2M1 element format, one shared scale per small block)     -> codecs
+ *  - "Online normalizer calculation for softmax" and "FlashAttention" (same
+ *    reference list): blockwise softmax with a running max and a running
+ *    sum.                                                         -> attn_fwd
+ *
+ * Fixed tiling of the method: Q blocks and KV blocks of 128 tokens; P is
+ * quantized once per KV block, after the running row max has been updated
+ * with that block; one E4M3 scale per 16 consecutive elements along the
+ * contraction dimension (d for Q and K, tokens for V and P).
+ *
+ * Readings where the pages are silent (each is restated where it is used):
+ *  R1 the K mean runs over the N real tokens of one (batch, head); summed in
+ *     fp64 in token order, divided by N in fp64, rounded once to fp32;
+ *  R2 K_s = fp32(K) - mean, one fp32 subtraction;
+ *  R3 block scale s = E4M3_RN_satfinite(fp32(amax / 6)); r = fp32(1 / s);
+ *     code = E2M1_RN_satfinite(fp32(x * r)); s == 0 gives all-zero codes;
+ *  R4 E2M1 and E4M3 round to nearest, ties to even, and keep the sign of a
+ *     value that rounds to zero (-0 -> code 0x8);
+ *  R5 packing: element 2i in the low nibble, element 2i+1 in the high one;
+ *  R6 V is quantized transposed: 16-token blocks per channel;
+ *  R7 raw Q is quantized (no Q smoothing); S is scaled by
+ *     c = fp32(sm_scale * log2(e)) in fp32 before the softmax, exp base 2;
+ *  R8 P = exp2(t - m_new) with m_new the running max including the current
+ *     block; the row sum l accumulates the unquantized P;
+ *  R9 columns >= N and, when causal, columns > row are -inf before the max.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define BLK 128   /* Q block and KV block, tokens */
+#define VEC 16    /* elements per E4M3 scale */
+
+/* ---------------------------------------------------------------- codecs */
+
+/* E2M1: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit, no inf/nan. */
+double oracle_e2m1_value(int code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/* E4M3 ("fn" variant): 1 sign, 4 exponent bits (bias 7), 3 mantissa bits;
+ * S.1111.111 is NaN, there is no infinity; largest finite value 448. */
+double oracle_e4m3_value(int code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp(m / 8.0, -6);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* Round to the nearest E2M1 magnitude, ties to the even code, saturating at
+ * 6; the sign bit is copied from x (reading R4).  Written as a search over
+ * the eight magnitudes so that it can be checked by eye. */
+int oracle_e2m1_rn(float x)
+{
+    double a = fabs((double)x);
+    /* saturation: at or above the largest magnitude the answer is 6 (for
+     * huge a the two distances below would compare equal in fp64) */
+    if (a >= 6.0) return (signbit(x) ? 8 : 0) | 7;
+    int best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        double dist = fabs(a - oracle_e2m1_value(c));
+        if (dist < bestd || (dist == bestd && (c & 1) == 0)) {
+            best = c;
+            bestd = dist;
+        }
+    }
+    return (signbit(x) ? 8 : 0) | best;
+}
+
+/* Round a non-negative value to the nearest finite E4M3 magnitude, ties to
+ * the even code, saturating at 448 (codes 0x00..0x7E). */
+int oracle_e4m3_rn_sat(float x)
+{
+    double a = fabs((double)x);
+    if (a >= 448.0) return 0x7E; /* saturation, as for E2M1 above */
+    int best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c < 127; ++c) {
+        double dist = fabs(a - oracle_e4m3_value(c));
+        if (dist < bestd || (dist == bestd && (c & 1) == 0)) {
+            best = c;
+            bestd = dist;
+        }
+    }
+    return best;
+}
+
+static float bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even (on the magnitude). */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x40);
+    uint32_t lo = u & 0xFFFF0000u;
+    uint32_t rem = u & 0xFFFFu;
+    uint32_t hi = lo + 0x10000u;
+    uint32_t r;
+    if (rem > 0x8000u) r = hi;
+    else if (rem < 0x8000u) r = lo;
+    else r = ((lo >> 16) & 1u) ? hi : lo;
+    return (uint16_t)(r >> 16);
+}
+
+/* Lookup tables filled once from the definitions above. */
+static float g_e2m1[16];
+static float g_e4m3[256];
+static int g_tables_ready = 0;
+
+static void tables_init(void)
+{
+    if (g_tables_ready) return;
+    for (int c = 0; c < 16; ++c) g_e2m1[c] = (float)oracle_e2m1_value(c);
+    for (int c = 0; c < 256; ++c) g_e4m3[c] = (float)oracle_e4m3_value(c);
+    g_tables_ready = 1;
+}
+
+/* One 16-element block (reading R3).  x holds n <= 16 values (missing
+ * tokens of a ragged last block are zeros and are passed as zeros).
+ * Writes 16 codes and returns the scale byte. */
+static int quant_block(const float *x, int *codes)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < VEC; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float ratio = amax / 6.0f;
+    int sc = oracle_e4m3_rn_sat(ratio);
+    float s = g_e4m3[sc];
+    if (s == 0.0f) {
+        for (int i = 0; i < VEC; ++i) codes[i] = 0;
+        return sc;
+    }
+    float r = 1.0f / s;
+    for (int i = 0; i < VEC; ++i) {
+        float y = x[i] * r;
+        codes[i] = oracle_e2m1_rn(y);
+    }
+    return sc;
+}
+
+int oracle_padded_len(int N) { return (N + BLK - 1) / BLK * BLK; }
+
+/* ------------------------------------------------------- K smoothing (R1) */
+
+void oracle_kmean(const uint16_t *k, int B, int H, int N, int d, float *mean)
+{
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int t = 0; t < N; ++t)
+                acc += (double)bf16_to_f32(k[(bh * N + t) * d + c]);
+            mean[bh * d + c] = (float)(acc / (double)N);
+        }
+    }
+}
+
+/* ----------------------------------------------------- quantization (R1-R6)
+ * Canonical layouts written here (N_p = N rounded up to 128):
+ *   q_codes, k_codes : [B*H][N_p][d/2]   bytes
+ *   q_sf, k_sf       : [B*H][N_p][d/16]  E4M3 bytes
+ *   vt_codes         : [B*H][d][N_p/2]   bytes (V transposed)
+ *   vt_sf            : [B*H][d][N_p/16]  E4M3 bytes
+ *   k_mean           : [B*H][d] fp32
+ * Padding tokens (t >= N) get code 0 and scale byte 0.
+ * smooth_k = 0 skips the subtraction (used to measure what smoothing buys). */
+void oracle_quantize_qkv(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         int B, int H, int N, int d, int smooth_k,
+                         uint8_t *q_codes, uint8_t *q_sf,
+                         uint8_t *k_codes, uint8_t *k_sf,
+                         uint8_t *vt_codes, uint8_t *vt_sf, float *k_mean)
+{
+    tables_init();
+    const long BH = (long)B * H;
+    const int Np = oracle_padded_len(N);
+    oracle_kmean(k, B, H, N, d, k_mean);
+
+    memset(q_codes, 0, (size_t)BH * Np * d / 2);
+    memset(k_codes, 0, (size_t)BH * Np * d / 2);
+    memset(q_sf, 0, (size_t)BH * Np * d / VEC);
+    memset(k_sf, 0, (size_t)BH * Np * d / VEC);
+    memset(vt_codes, 0, (size_t)BH * d * Np / 2);
+    memset(vt_sf, 0, (size_t)BH * d * Np / VEC);
+
+#pragma omp parallel for schedule(dynamic)
+    for (long bh = 0; bh < BH; ++bh) {
+        float x[VEC];
+        int codes[VEC];
+        /* Q and K: blocks of 16 along d, per token. */
+        for (int t = 0; t < N; ++t) {
+            for (int b = 0; b < d / VEC; ++b) {
+                /* Q */
+                for (int i = 0; i < VEC; ++i)
+                    x[i] = bf16_to_f32(q[(bh * N + t) * d + b * VEC + i]);
+                int sc = quant_block(x, codes);
+                q_sf[(bh * Np + t) * (d / VEC) + b] = (uint8_t)sc;
+                for (int i = 0; i < VEC; i += 2)
+                    q_codes[(bh * Np + t) * (d / 2) + (b * VEC + i) / 2] =
+                        (uint8_t)(codes[i] | (codes[i + 1] << 4));
+                /* K, smoothed (R2) */
+                for (int i = 0; i < VEC; ++i) {
+                    float kv = bf16_to_f32(k[(bh * N + t) * d + b * VEC + i]);
+                    x[i] = smooth_k ? kv - k_mean[bh * d + b * VEC + i] : kv;
+                }
+                sc = quant_block(x, codes);
+                k_sf[(bh * Np + t) * (d / VEC) + b] = (uint8_t)sc;
+                for (int i = 0; i < VEC; i += 2)
+                    k_codes[(bh * Np + t) * (d / 2) + (b * VEC + i) / 2] =
+                        (uint8_t)(codes[i] | (codes[i + 1] << 4));
+            }
+        }
+        /* V: blocks of 16 tokens, per channel (R6). */
+        for (int c = 0; c < d; ++c) {
+            for (int tb = 0; tb < Np / VEC; ++tb) {
+                for (int i = 0; i < VEC; ++i) {
+                    int t = tb * VEC + i;
+                    x[i] = (t < N) ? bf16_to_f32(v[(bh * N + t) * d + c]) : 0.0f;
+                }
+                int sc = quant_block(x, codes);
+                vt_sf[(bh * d + c) * (Np / VEC) + tb] = (uint8_t)sc;
+                for (int i = 0; i < VEC; i += 2)
+                    vt_codes[(bh * d + c) * (Np / 2) + (tb * VEC + i) / 2] =
+                        (uint8_t)(codes[i] | (codes[i + 1] << 4));
+            }
+        }
+    }
+}
+
+/* Dequantize one packed element. */
+static double deq(const uint8_t *codes, const uint8_t *sf, long elem, long sf_idx)
+{
+    uint8_t byte = codes[elem >> 1];
+    int code = (elem & 1) ? (byte >> 4) : (byte & 15);
+    return (double)g_e2m1[code] * (double)g_e4m3[sf[sf_idx]];
+}
+
+/* ------------------------------------------------- tiled attention (R7-R9)
+ * units: n_units pairs (bh, q_block); NULL means every (bh, q_block).
+ * out: bf16 [B*H][N][d]; only rows of the listed units are written. */
+void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
+                     const uint8_t *k_codes, const uint8_t *k_sf,
+                     const uint8_t *vt_codes, const uint8_t *vt_sf,
+                     int B, int H, int N, int d, int causal, float sm_scale,
+                     const int32_t *units, int n_units, uint16_t *out)
+{
+    tables_init();
+    const long BH = (long)B * H;
+    const int Np = oracle_padded_len(N);
+    const int nqb = Np / BLK;
+    const float c_log2 = (float)((double)sm_scale * 1.4426950408889634);
+    const long total = units ? n_units : BH * nqb;
+
+#pragma omp parallel for schedule(dynamic)
+    for (long u = 0; u < total; ++u) {
+        long bh = units ? units[2 * u] : u / nqb;
+        int qb = units ? units[2 * u + 1] : (int)(u % nqb);
+        int nkv = causal ? qb + 1 : Np / BLK;
+        int ncol = nkv * BLK;
+        /* Dequantized operands of this (batch, head), cached so that each
+         * value is decoded once; the sums below are unchanged by this. */
+        double *qrow = (double *)malloc(sizeof(double) * d);
+        double *khat = (double *)malloc(sizeof(double) * (size_t)ncol * d);
+        double *vhat = (double *)malloc(sizeof(double) * (size_t)ncol * d);
+        float *O = (float *)malloc(sizeof(float) * d);
+        float t[BLK], p[BLK], phat[BLK];
+        int codes[VEC];
+        for (int col = 0; col < ncol; ++col)
+            for (int c = 0; c < d; ++c)
+                khat[(size_t)col * d + c] = deq(k_codes, k_sf, (bh * Np + col) * d + c,
+                                                (bh * Np + col) * (d / VEC) + c / VEC);
+        for (int c = 0; c < d; ++c)
+            for (int col = 0; col < ncol; ++col)
+                vhat[(size_t)c * ncol + col] = deq(vt_codes, vt_sf, (bh * d + c) * Np + col,
+                                                   (bh * d + c) * (Np / VEC) + col / VEC);
+
+        for (int row = qb * BLK; row < qb * BLK + BLK && row < N; ++row) {
+            for (int c = 0; c < d; ++c)
+                qrow[c] = deq(q_codes, q_sf, (bh * Np + row) * d + c,
+                              (bh * Np + row) * (d / VEC) + c / VEC);
+            float m = -INFINITY, l = 0.0f;
+            for (int c = 0; c < d; ++c) O[c] = 0.0f;
+
+            for (int j = 0; j < nkv; ++j) {
+                /* S row for this KV block: exact fp64 dot, rounded once. */
+                float bmax = -INFINITY;
+                for (int i = 0; i < BLK; ++i) {
+                    int col = j * BLK + i;
+                    if (col >= N || (causal && col > row)) { t[i] = -INFINITY; continue; }
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        acc += qrow[c] * khat[(size_t)col * d + c];
+                    float s = (float)acc;
+                    t[i] = s * c_log2;
+                    if (t[i] > bmax) bmax = t[i];
+                }
+                /* Online softmax update. */
+                float m_new = m > bmax ? m : bmax;
+                float alpha, rowsum;
+                if (m_new == -INFINITY) { /* fully masked so far (R9 guard) */
+                    alpha = 1.0f;
+                    for (int i = 0; i < BLK; ++i) p[i] = 0.0f;
+                } else {
+                    alpha = exp2f(m - m_new);
+                    for (int i = 0; i < BLK; ++i) p[i] = exp2f(t[i] - m_new);
+                }
+                double psum = 0.0;
+                for (int i = 0; i < BLK; ++i) psum += p[i];
+                rowsum = (float)psum;
+                l = alpha * l + rowsum;
+                /* Quantize P per 16-column block (R3, R8). */
+                for (int b = 0; b < BLK / VEC; ++b) {
+                    int sc = quant_block(p + b * VEC, codes);
+                    for (int i = 0; i < VEC; ++i)
+                        phat[b * VEC + i] = g_e2m1[codes[i]] * g_e4m3[sc];
+                }
+                /* O = alpha * O + P^ V^ (exact fp64 sum, rounded once). */
+                for (int c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (int i = 0; i < BLK; ++i)
+                        acc += (double)phat[i] * vhat[(size_t)c * ncol + j * BLK + i];
+                    O[c] = alpha * O[c] + (float)acc;
+                }
+                m = m_new;
+            }
+            for (int c = 0; c < d; ++c)
+                out[(bh * N + row) * d + c] = oracle_f32_to_bf16(O[c] / l);
+        }
+        free(qrow);
+        free(khat);
+        free(vhat);
+        free(O);
+    }
+}
+
+/* --------------------------------------------- exact attention (fp64)
+ * softmax(Q K^T * sm_scale) V on the bf16 inputs, no quantization.  k_sub,
+ * if not NULL, is subtracted from K first (fp32 [B*H][d]); this is how the
+ * smoothing invariance is checked.  Rows of the listed units only. */
+void oracle_attn_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       int B, int H, int N, int d, int causal, float sm_scale,
+                       const float *k_sub, const int32_t *units, int n_units,
+                       double *out)
+{
+    const long BH = (long)B * H;
+    const int nqb = oracle_padded_len(N) / BLK;
+    const long total = units ? n_units : BH * nqb;
+
+#pragma omp parallel for schedule(dynamic)
+    for (long u = 0; u < total; ++u) {
+        long bh = units ? units[2 * u] : u / nqb;
+        int qb = units ? units[2 * u + 1] : (int)(u % nqb);
+        double *logit = (double *)malloc(sizeof(double) * N);
+        for (int row = qb * BLK; row < qb * BLK + BLK && row < N; ++row) {
+            int ncol = causal ? row + 1 : N;
+            double mx = -INFINITY;
+            for (int col = 0; col < ncol; ++col) {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    double kk = bf16_to_f32(k[(bh * N + col) * d + c]);
+                    if (k_sub) kk -= (double)k_sub[bh * d + c];
+                    acc += (double)bf16_to_f32(q[(bh * N + row) * d + c]) * kk;
+                }
+                logit[col] = acc * (double)sm_scale;
+                if (logit[col] > mx) mx = logit[col];
+            }
+            double den = 0.0;
+            for (int col = 0; col < ncol; ++col) {
+                logit[col] = exp(logit[col] - mx);
+                den += logit[col];
+            }
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int col = 0; col < ncol; ++col)
+                    acc += logit[col] * (double)bf16_to_f32(v[(bh * N + col) * d + c]);
+                out[(bh * N + row) * d + c] = acc / den;
+            }
+        }
+        free(logit);
+    }
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
