@@ -1,0 +1,346 @@
+#!/usr/bin/env python3
+"""Throughput of libsa3 (microscaled-FP4 attention forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sa3|reference]
+
+One step = the whole hot path on one batch: sa3_quantize_qkv (K smoothing
++ FP4 microscaling of Q, K, V) followed by sa3_attn_fwd, on the non-causal
+workload B=2, H=16, N=4096, d=128 (seeded synthetic bf16 inputs already
+resident in HBM).  The metric is attention TOPS = 4*B*H*N^2*d / t.
+L2 is flushed (256 MiB write) before every timed step; each step is timed
+with CUDA events on the launching stream, with a barrier and a device
+synchronize around the K timed steps; multi-GPU runs take the maximum
+over ranks and report the whole-job rate (every rank runs its own batch:
+weak scaling, no data-path collective).
+
+--impl reference runs the CPU oracle (oracle/) as it stands on the host
+cores, on a bounded sample of the same workload, and prints the same line
+with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sa3_inputs  # noqa: E402
+
+WORKLOAD = "noncausal_b2h16n4096d128"
+METRIC = "attention TOPS (4*B*H*N^2*d/t) and % of B200 dense FP4 peak, 1 GPU"
+UNIT = "TOPS"
+FP4_DATASHEET_TOPS = 9000.0        # NVIDIA B200 dense FP4 (18 PF with 2:4 sparsity)
+FP4_PER_BF16 = 4.0                 # nominal dense FP4 / bf16 ratio (9 / 2.25 PF)
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sa3", choices=["sa3", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=list(sa3_inputs.WORKLOADS))
+    ap.add_argument("--skip-cpu-baseline", action="store_true",
+                    help="omit the oracle timing (for profiler runs)")
+    return ap.parse_args()
+
+
+def dist_init(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n:
+        raise SystemExit(f"--gpus {n} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                             timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"bf16_tflops": FALLBACK_BF16_TFLOPS, "bf16_tflops_sustained": 1400.0,
+                "hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_sa3(args, rank, world, local):
+    import bit_quantized_attention_sa3_b200 as sa3
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = sa3_inputs.WORKLOADS[args.workload]
+    B, H, N, d, causal = w.B, w.H, w.N, w.d, w.causal
+    q_h, k_h, v_h = sa3_inputs.make_qkv(w, seed=rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    qz = sa3.empty_quantized(B, H, N, d, dev)
+    ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sa3.quantize_qkv(q, k, v, out=qz, workspace=ws)
+        sa3.attn_fwd(qz, causal=causal, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if sa3.device_status() != sa3.SA3_OK:
+        raise RuntimeError("device wait gave up during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)                   # evict the previous step from L2
+            ev[i][0].record(stream)
+            sa3.quantize_qkv(q, k, v, out=qz, workspace=ws)
+            ev[i][1].record(stream)
+            sa3.attn_fwd(qz, causal=causal, out=out)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    if sa3.device_status() != sa3.SA3_OK:
+        raise RuntimeError("device wait gave up during the timed steps")
+
+    # end-to-end through the public API: pinned host in -> host out
+    qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    out_h = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(qp, non_blocking=True)
+        kd.copy_(kp, non_blocking=True)
+        vd.copy_(vp, non_blocking=True)
+        sa3.quantize_qkv(qd, kd, vd, out=qz, workspace=ws)
+        sa3.attn_fwd(qz, causal=causal, out=out)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 2)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+
+    def gmax(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    t_step = gmax(sum(step_ms) / len(step_ms))
+    t_quant = gmax(sum(quant_ms) / len(quant_ms))
+    t_attn = gmax(sum(attn_ms) / len(attn_ms))
+    t_e2e = gmax(e2e_ms)
+    if rank != 0:
+        return
+    pk, src = peaks()
+    ops = w.ops
+    fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
+    achieved = ops / (t_attn * 1e-3) / 1e12
+    qk_bytes = 3 * (B * H * N * d * 2) + 3 * (B * H * sa3.padded_len(N) * d // 2) \
+        + 3 * (B * H * sa3.padded_len(N) * d // 16)
+    line = {
+        "metric": METRIC,
+        "value": round(world * ops / (t_step * 1e-3) / 1e12, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp4-e2m1 (ue4m3 scales, fp32 accumulate)",
+        "data": "synthetic (seeded, sa3_inputs.py)",
+        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                   "step": "sa3_quantize_qkv + sa3_attn_fwd", "l2": "flushed (256 MiB write) before each step",
+                   "parallelism": f"{world} independent replicas (one batch per GPU)"},
+        "attn_only": {"value": round(achieved, 2), "unit": UNIT, "ms": round(t_attn, 4),
+                      "frac_of_datasheet_fp4_9000": round(achieved / FP4_DATASHEET_TOPS, 4)},
+        "quantize": {"ms": round(t_quant, 4), "GB_per_s": round(qk_bytes / (t_quant * 1e-3) / 1e9, 1),
+                     "algorithmic_bytes": qk_bytes},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4), "traffic": None,
+                     "kernel": "attn_fwd_kernel<128>",
+                     "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"},
+        "e2e": {"value": round(world * ops / (t_e2e * 1e-3) / 1e12, 2), "unit": UNIT, "ms": round(t_e2e, 4),
+                "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 2},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.skip_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None):
+    """The oracle, as it stands, on the host cores: full quantization plus
+    attention for a seeded sample of Q blocks; the full-job time is
+    extrapolated from the sampled blocks (non-causal: every block costs
+    the same)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    qz = oracle.quantize_qkv(q, k, v)
+    t_quant = time.perf_counter() - t0
+    nqb = (w.N + 127) // 128
+    total_units = w.B * w.H * nqb
+    rng = np.random.default_rng(0)
+    order = rng.permutation(total_units)
+    done, t_attn, n = 0, 0.0, 8
+    while True:
+        chunk = order[done:done + n]
+        if len(chunk) == 0:
+            break
+        units = [(int(u) // nqb, int(u) % nqb) for u in chunk]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qz, w.N, w.causal, units=units)
+        t_attn += time.perf_counter() - t0
+        done += len(chunk)
+        if t_quant + t_attn > budget_s or (units_cap and done >= units_cap):
+            break
+        n = min(4 * n, 256)
+    if w.causal:
+        weights = np.array([(u % nqb) + 1 for u in range(total_units)], float)
+        frac = weights[order[:done]].sum() / weights.sum()
+    else:
+        frac = done / total_units
+    t_full = t_quant + t_attn / frac
+    return {"value": round(w.ops / t_full / 1e12, 6), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"full quantization ({t_quant:.2f} s) + attention for {done} of {total_units} "
+                       f"Q blocks ({t_attn:.2f} s), extrapolated to the whole {w.name} job "
+                       f"({t_full:.1f} s)")}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = sa3_inputs.WORKLOADS[args.workload]
+    q, k, v = sa3_inputs.make_qkv(w, seed=0)
+    per_step = []
+    budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, q, k, v, budget_s=budget)
+        if i >= args.warmup:
+            per_step.append(cb)
+    vals = [c["value"] for c in per_step]
+    value = statistics.mean(vals)
+    last = per_step[-1]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(w.ops / (value * 1e12) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)",
+        "data": "synthetic (seeded, sa3_inputs.py)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "step": "oracle quantize + tiled attention (sampled, extrapolated)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_sa3(args, rank, world, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+"""libsa3 Python binding: microscaled-FP4 attention forward on B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels of ``libsa3.so`` (C ABI in ``include/sa3.h``); PyTorch provides the
+device memory and the current stream.  There is no CPU fallback: if the
+library is missing or a call fails, an exception is raised.
+
+    qz = quantize_qkv(q, k, v)          # K smoothing + FP4 microscaling
+    out = attn_fwd(qz, causal=False)    # FP4 attention, bf16 out
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa3.so")
+
+SA3_OK = 0
+SA3_ERR_INVALID_ARG = 1
+SA3_ERR_UNSUPPORTED = 2
+SA3_ERR_CUDA = 3
+SA3_ERR_TIMEOUT = 4
+_NAMES = {0: "SA3_OK", 1: "SA3_ERR_INVALID_ARG", 2: "SA3_ERR_UNSUPPORTED", 3: "SA3_ERR_CUDA",
+          4: "SA3_ERR_TIMEOUT"}
+
+BLK = 128
+
+
+class Sa3Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {_NAMES.get(code, code)}")
+        self.code = code
+
+
+class _QKV(ctypes.Structure):
+    _fields_ = [("q_fp4", ctypes.c_void_p), ("q_sf", ctypes.c_void_p),
+                ("k_fp4", ctypes.c_void_p), ("k_sf", ctypes.c_void_p),
+                ("vt_fp4", ctypes.c_void_p), ("vt_sf", ctypes.c_void_p),
+                ("k_mean", ctypes.c_void_p)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsa3.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m bit_quantized_attention_sa3_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            L.sa3_version.restype = ctypes.c_char_p
+            L.sa3_version.argtypes = []
+            L.sa3_quantize_qkv.restype = I
+            L.sa3_quantize_qkv.argtypes = [P, P, P, I, I, I, I, ctypes.POINTER(_QKV), P, ctypes.c_size_t, P]
+            L.sa3_attn_fwd.restype = I
+            L.sa3_attn_fwd.argtypes = [ctypes.POINTER(_QKV), I, I, I, I, I, F, P, P]
+            L.sa3_device_status.restype = I
+            L.sa3_device_status.argtypes = [P]
+            _lib = L
+    return _lib
+
+
+def version() -> str:
+    return lib().sa3_version().decode()
+
+
+# ---------------------------------------------------------------- sizes
+def padded_len(N: int) -> int:
+    return (N + BLK - 1) // BLK * BLK
+
+
+def quant_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return B * H * ((N + 511) // 512) * d * 8
+
+
+@dataclasses.dataclass
+class QuantizedQKV:
+    """Device buffers of the quantized operands (layouts: include/sa3.h)."""
+    q_fp4: torch.Tensor   # u8 [B,H,Np,d/2]
+    q_sf: torch.Tensor    # u8, 128x4 scale atoms
+    k_fp4: torch.Tensor   # u8 [B,H,Np,d/2]
+    k_sf: torch.Tensor
+    vt_fp4: torch.Tensor  # u8 [B,H,d,Np/2]
+    vt_sf: torch.Tensor
+    k_mean: torch.Tensor  # f32 [B,H,d]
+    B: int
+    H: int
+    N: int
+    d: int
+
+    def struct(self) -> _QKV:
+        return _QKV(self.q_fp4.data_ptr(), self.q_sf.data_ptr(), self.k_fp4.data_ptr(),
+                    self.k_sf.data_ptr(), self.vt_fp4.data_ptr(), self.vt_sf.data_ptr(),
+                    self.k_mean.data_ptr())
+
+
+def empty_quantized(B: int, H: int, N: int, d: int, device="cuda") -> QuantizedQKV:
+    Np = padded_len(N)
+    u8 = dict(dtype=torch.uint8, device=device)
+    return QuantizedQKV(
+        q_fp4=torch.empty((B, H, Np, d // 2), **u8), q_sf=torch.empty(B * H * Np * d // 16, **u8),
+        k_fp4=torch.empty((B, H, Np, d // 2), **u8), k_sf=torch.empty(B * H * Np * d // 16, **u8),
+        vt_fp4=torch.empty((B, H, d, Np // 2), **u8), vt_sf=torch.empty(B * H * Np * 8, **u8),
+        k_mean=torch.empty((B, H, d), dtype=torch.float32, device=device), B=B, H=H, N=N, d=d)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check_input(t: torch.Tensor, name: str):
+    if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+        raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor [B,H,N,d]")
+
+
+def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 out: QuantizedQKV | None = None, workspace: torch.Tensor | None = None,
+                 stream=None) -> QuantizedQKV:
+    """sa3_quantize_qkv: K smoothing, then E2M1 codes + E4M3 scales of Q, K, V."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_input(t, n)
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape (self-attention)")
+    B, H, N, d = q.shape
+    if out is None:
+        out = empty_quantized(B, H, N, d, q.device)
+    nbytes = quant_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    st = out.struct()
+    rc = lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(st),
+                                workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if rc != SA3_OK:
+        raise Sa3Error(rc, "sa3_quantize_qkv")
+    return out
+
+
+def attn_fwd(qz: QuantizedQKV, causal: bool = False, sm_scale: float | None = None,
+             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """sa3_attn_fwd: FP4 attention of quantized operands; bf16 [B,H,N,d]."""
+    B, H, N, d = qz.B, qz.H, qz.N, qz.d
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=qz.q_fp4.device)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    st = qz.struct()
+    rc = lib().sa3_attn_fwd(ctypes.byref(st), B, H, N, d, int(bool(causal)), float(sm_scale),
+                            out.data_ptr(), _stream_ptr(stream))
+    if rc != SA3_OK:
+        raise Sa3Error(rc, "sa3_attn_fwd")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronizes the stream; SA3_ERR_TIMEOUT if a bounded wait gave up."""
+    return lib().sa3_device_status(_stream_ptr(stream))
+
+
+def sa3_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                  sm_scale: float | None = None) -> torch.Tensor:
+    """Plug-in attention: quantize then attend; bf16 [B,H,N,d] in and out."""
+    return attn_fwd(quantize_qkv(q, k, v), causal=causal, sm_scale=sm_scale)

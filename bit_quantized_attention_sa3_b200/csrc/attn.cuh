@@ -1,0 +1,478 @@
+// attn.cuh -- microscaled-FP4 attention forward for sm_100a.
+//
+// Method ("SageAttention3: Microscaling FP4 Attention ...", abstract; the
+// blockwise softmax of "Online normalizer calculation for softmax" and
+// FlashAttention, both in its reference list): per 128-row Q block and
+// 128-token KV block j,
+//   S = Q^ K^_j^T                      block-scaled FP4 MMA, fp32 in TMEM
+//   t = S*c, m' = max(m, rowmax t), alpha = 2^(m-m'), P = 2^(t-m')
+//   l = alpha*l + rowsum P; P^ = E2M1/E4M3 microscaled P (per 16 columns)
+//   O = alpha*O + P^ V^_j              block-scaled FP4 MMA, fp32 in TMEM
+// and finally out = bf16(O / l).
+//
+// One CTA = two 128-row Q tiles of one (b, h), 12 warps:
+//   warps 0-3  softmax for Q tile 0 (one thread per row = one TMEM lane)
+//   warps 4-7  softmax for Q tile 1
+//   warp  8    producer: TMA loads of Q, and of K / V^T codes + scales into
+//              a 3-stage ring (mbarrier transaction counts)
+//   warp  9    allocates TMEM and issues every tcgen05 op from one thread:
+//              scale-factor copies (tcgen05.cp), S = Q K^T, O += P V
+//   warps 10-11 idle (registers are granted per warpgroup)
+// TMEM (512 columns): S (128, shared by both tiles -- each softmax group
+// loads it to registers at once and releases it), O0, O1 (d each), and
+// the scale factors of Q0, Q1, K, P and V.  tcgen05.cp and tcgen05.mma
+// from one thread execute in issue order, so each scale-factor region is
+// rewritten right before the MMA that reads it.  P goes through shared
+// memory (64-byte swizzled K-major rows + 512-byte scale atoms) because
+// the block-scaled FP4 MMA takes A from shared memory only.
+// The tensor pipe order per KV block j is QK0(j+1), PV0(j), QK1(j+1),
+// PV1(j): each softmax group finds its next S ready as soon as it has
+// produced its P, so the two groups run concurrently and the exp / FMA
+// pipes (the bottleneck on B200) stay busy.
+#pragma once
+
+#include "sa3_internal.h"
+#include "sm100.cuh"
+
+namespace sa3 {
+namespace attn {
+
+constexpr int kBlk = 128;
+constexpr int kStages = 3;
+constexpr int kThreads = 384;  // three warpgroups, 168 registers per thread
+
+template <int D>
+struct Cfg {
+    static constexpr int al(int x) { return (x + 1023) & ~1023; }
+    static constexpr int kRowB = D / 2;                 // bytes per Q/K code row
+    static constexpr int kQBytes = kBlk * kRowB;
+    static constexpr int kSfBytes = (D / 64) * 512;    // Q or K tile scales
+    static constexpr int kVBytes = D * 64;             // V^T tile: D rows x 128 tokens
+    static constexpr int kVsfBytes = 1024;
+    static constexpr int kPBytes = kBlk * 64;
+    static constexpr int kPsfBytes = 1024;
+    static constexpr uint32_t kQKLayout = (D == 128) ? 4u : 6u;  // 64B / 32B swizzle
+    static constexpr uint32_t kQKSbo = 8 * kRowB;
+    // shared memory map, offsets from a 1024-byte aligned base
+    static constexpr int oQ0 = 0;
+    static constexpr int oQ1 = al(oQ0 + kQBytes);
+    static constexpr int oQsf0 = al(oQ1 + kQBytes);
+    static constexpr int oQsf1 = oQsf0 + kSfBytes;
+    static constexpr int oStage = al(oQsf1 + kSfBytes);
+    static constexpr int sK = 0;
+    static constexpr int sV = al(kQBytes);
+    static constexpr int sKsf = sV + al(kVBytes);
+    static constexpr int sVsf = sKsf + kSfBytes;
+    static constexpr int kStageBytes = al(sVsf + kVsfBytes);
+    static constexpr int oP0 = oStage + kStages * kStageBytes;
+    static constexpr int oP1 = oP0 + kPBytes;
+    static constexpr int oPsf0 = oP1 + kPBytes;
+    static constexpr int oPsf1 = oPsf0 + kPsfBytes;
+    static constexpr int oBar = oPsf1 + kPsfBytes;
+    static constexpr int kSmemBytes = oBar + 256 + 1024;
+    // TMEM columns
+    static constexpr uint32_t tS = 0;
+    static constexpr uint32_t tO0 = 128;
+    static constexpr uint32_t tO1 = 128 + D;
+    static constexpr uint32_t tSfq0 = 128 + 2 * D;
+    static constexpr uint32_t tSfq1 = tSfq0 + 4 * (D / 64);
+    static constexpr uint32_t tSfk = tSfq1 + 4 * (D / 64);
+    static constexpr uint32_t tSfp = tSfk + 4 * (D / 64);
+    static constexpr uint32_t tSfv = tSfp + 8;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(tSfv + 8 <= kTmemCols, "TMEM budget");
+};
+
+// Barrier slots (uint64 each) after oBar.
+enum : int {
+    kBarQ = 0,
+    kBarKvFull = 1,                  // kStages
+    kBarKvEmpty = 1 + kStages,       // kStages
+    kBarSFull = 1 + 2 * kStages,     // 2
+    kBarSEmpty = 3 + 2 * kStages,    // 1
+    kBarPFull = 4 + 2 * kStages,     // 2
+    kBarPvDone = 6 + 2 * kStages,    // 2
+    kBarDrain = 8 + 2 * kStages,     // 1
+    kBarCount = 9 + 2 * kStages
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// mbar_wait with a warp-uniform result, for code that continues with
+// .sync.aligned tcgen05 instructions.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    const bool ok = mbar_wait(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag (used to drain copies in
+// flight before the CTA exits).
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicOr(&g_sa3_status, 1u);
+            return;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t *base = smem_raw + (base_s - raw_s);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + C::oBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kBarCount);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int nqt = p.Np / kBlk;
+    // causal: heaviest Q-tile pairs first
+    const int pair = p.causal ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
+                              : static_cast<int>(blockIdx.x);
+    const int tile0 = 2 * pair;
+    const int tile1 = 2 * pair + 1;
+    const bool valid1 = tile1 < nqt;
+    const int n0 = p.causal ? tile0 + 1 : nqt;
+    const int n1 = valid1 ? (p.causal ? tile1 + 1 : nqt) : 0;
+    const int nmax = n0 > n1 ? n0 : n1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars + kBarQ, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bars + kBarKvFull + s, 1);
+            mbar_init(bars + kBarKvEmpty + s, 1);
+        }
+        mbar_init(bars + kBarSFull + 0, 1);
+        mbar_init(bars + kBarSFull + 1, 1);
+        mbar_init(bars + kBarSEmpty, 128);
+        mbar_init(bars + kBarPFull + 0, 128);
+        mbar_init(bars + kBarPFull + 1, 128);
+        mbar_init(bars + kBarPvDone + 0, 1);
+        mbar_init(bars + kBarPvDone + 1, 1);
+        mbar_init(bars + kBarDrain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= 8) {
+      if (warp == 8) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            uint64_t *bq = bars + kBarQ;
+            mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * (C::kQBytes + C::kSfBytes));
+            tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Np + tile0 * kBlk, bq);
+            bulk_load(base + C::oQsf0, p.q_sf + static_cast<size_t>(bh * nqt + tile0) * C::kSfBytes, C::kSfBytes, bq);
+            if (valid1) {
+                tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Np + tile1 * kBlk, bq);
+                bulk_load(base + C::oQsf1, p.q_sf + static_cast<size_t>(bh * nqt + tile1) * C::kSfBytes, C::kSfBytes,
+                          bq);
+            }
+            int issued = 0;
+            for (int j = 0; j < nmax; ++j) {
+                const int s = j % kStages;
+                const int u = j / kStages;
+                if (u > 0 && !mbar_wait(bars + kBarKvEmpty + s, (u - 1) & 1, abort_flag)) break;
+                uint8_t *st = base + C::oStage + s * C::kStageBytes;
+                uint64_t *bf = bars + kBarKvFull + s;
+                mbar_arrive_expect_tx(bf, C::kQBytes + C::kSfBytes + C::kVBytes + C::kVsfBytes);
+                tma_load_2d(st + C::sK, &tm_k, 0, bh * p.Np + j * kBlk, bf);
+                bulk_load(st + C::sKsf, p.k_sf + static_cast<size_t>(bh * nqt + j) * C::kSfBytes, C::kSfBytes, bf);
+                tma_load_2d(st + C::sV, &tm_v, j * 64, bh * D, bf);
+                bulk_load(st + C::sVsf, p.vt_sf + (static_cast<size_t>(bh) * (p.Np / 64) + 2 * j) * 512, C::kVsfBytes,
+                          bf);
+                issued = j + 1;
+            }
+            // Let every copy this thread started land before the CTA exits.
+            drain_wait(bq, 0);
+            for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
+                drain_wait(bars + kBarKvFull + j % kStages, (j / kStages) & 1);
+        }
+    } else if (warp == 9) {
+        // ----------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_mxf4nvf4(128, 128);
+            constexpr uint32_t idesc_pv = idesc_mxf4nvf4(128, D);
+            int nqk = 0;
+            auto stage_s = [&](int j) -> uint32_t {
+                return base_s + C::oStage + static_cast<uint32_t>(j % kStages) * C::kStageBytes;
+            };
+            auto copy_ksf = [&](int j) {
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a)
+                    tc_cp_32x128b_warpx4(tmem + C::tSfk + 4 * a, sdesc_sf_atom(stage_s(j) + C::sKsf + 512 * a));
+            };
+            auto issue_qk = [&](int i, int j) -> bool {
+                if (nqk > 0 && !mbar_wait(bars + kBarSEmpty, (nqk - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t qa = base_s + (i ? C::oQ1 : C::oQ0);
+                const uint32_t kb = stage_s(j) + C::sK;
+#pragma unroll
+                for (int kc = 0; kc < D / 64; ++kc)
+                    tc_mma_mxf4nvf4(tmem + C::tS, sdesc_kmajor_sw(qa + 32 * kc, C::kQKSbo, C::kQKLayout),
+                                    sdesc_kmajor_sw(kb + 32 * kc, C::kQKSbo, C::kQKLayout), idesc_qk,
+                                    tmem + (i ? C::tSfq1 : C::tSfq0) + 4 * kc, tmem + C::tSfk + 4 * kc, kc > 0);
+                tc_commit(bars + kBarSFull + i);
+                ++nqk;
+                return true;
+            };
+            auto issue_pv = [&](int i, int j, bool load_vsf) -> bool {
+                if (!mbar_wait(bars + kBarPFull + i, j & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t pa = base_s + (i ? C::oP1 : C::oP0);
+                const uint32_t psf = base_s + (i ? C::oPsf1 : C::oPsf0);
+                const uint32_t vb = stage_s(j) + C::sV;
+                const uint32_t vsf = stage_s(j) + C::sVsf;
+                tc_cp_32x128b_warpx4(tmem + C::tSfp, sdesc_sf_atom(psf));
+                tc_cp_32x128b_warpx4(tmem + C::tSfp + 4, sdesc_sf_atom(psf + 512));
+                if (load_vsf) {
+                    tc_cp_32x128b_warpx4(tmem + C::tSfv, sdesc_sf_atom(vsf));
+                    tc_cp_32x128b_warpx4(tmem + C::tSfv + 4, sdesc_sf_atom(vsf + 512));
+                }
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc)
+                    tc_mma_mxf4nvf4(tmem + (i ? C::tO1 : C::tO0), sdesc_kmajor_sw(pa + 32 * kc, 512, 4u),
+                                    sdesc_kmajor_sw(vb + 32 * kc, 512, 4u), idesc_pv, tmem + C::tSfp + 4 * kc,
+                                    tmem + C::tSfv + 4 * kc, (j > 0 || kc > 0) ? 1u : 0u);
+                tc_commit(bars + kBarPvDone + i);
+                return true;
+            };
+
+            bool ok = mbar_wait(bars + kBarQ, 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    tc_cp_32x128b_warpx4(tmem + C::tSfq0 + 4 * a, sdesc_sf_atom(base_s + C::oQsf0 + 512 * a));
+                    if (valid1)
+                        tc_cp_32x128b_warpx4(tmem + C::tSfq1 + 4 * a, sdesc_sf_atom(base_s + C::oQsf1 + 512 * a));
+                }
+                ok = mbar_wait(bars + kBarKvFull + 0, 0, abort_flag);
+            }
+            if (ok) {
+                tc_fence_after();
+                copy_ksf(0);
+                if (n0 > 0) ok = issue_qk(0, 0);
+                if (ok && n1 > 0) ok = issue_qk(1, 0);
+            }
+            for (int j = 0; ok && j < nmax; ++j) {
+                if (j + 1 < nmax) {
+                    ok = mbar_wait(bars + kBarKvFull + (j + 1) % kStages, ((j + 1) / kStages) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    copy_ksf(j + 1);
+                }
+                if (j + 1 < n0 && !(ok = issue_qk(0, j + 1))) break;
+                if (j < n0 && !(ok = issue_pv(0, j, true))) break;
+                if (j + 1 < n1 && !(ok = issue_qk(1, j + 1))) break;
+                if (j < n1 && !(ok = issue_pv(1, j, !(j < n0)))) break;
+                tc_commit(bars + kBarKvEmpty + j % kStages);
+            }
+            // Every tcgen05 op issued above completes before TMEM is freed.
+            tc_commit(bars + kBarDrain);
+            drain_wait(bars + kBarDrain, 0);
+        }
+        __syncwarp();
+      }
+    } else {
+        // ------------------------------------------------------- softmax
+        const int i = warp >> 2;       // Q tile of this warpgroup
+        const int wq = warp & 3;       // TMEM sub-partition = rows 32*wq ..
+        const int r = wq * 32 + lane;  // row inside the tile
+        const int tile = i ? tile1 : tile0;
+        const int grow = tile * kBlk + r;
+        const int n_i = i ? n1 : n0;
+        const float c2 = p.scale_log2;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t tO = i ? C::tO1 : C::tO0;
+        uint8_t *P = base + (i ? C::oP1 : C::oP0);
+        uint8_t *Psf = base + (i ? C::oPsf1 : C::oPsf0);
+        float m = -INFINITY;
+        float l = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < n_i; ++j) {
+            if (!warp_wait(bars + kBarSFull + i, j & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t s[4][32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tmem_ld32(trow + C::tS + 32 * q, s[q]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) reg_fence32(s[q]);
+            tc_fence_before();
+            mbar_arrive(bars + kBarSEmpty);
+
+            const int col0 = j * kBlk;
+            const bool tail = col0 + kBlk > p.N;
+            const bool diag = p.causal && (col0 + kBlk - 1 > tile * kBlk);
+            if (tail || diag) {
+                // columns col0 + k with k >= lim are masked for this row
+                int lim = p.N - col0;
+                if (p.causal) lim = min(lim, grow - col0 + 1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * q + e >= lim) s[q][e] = __float_as_uint(-INFINITY);
+                }
+            }
+            float bm[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                float mx = __uint_as_float(s[b >> 1][(b & 1) * 16]);
+#pragma unroll
+                for (int e = 1; e < 16; ++e) mx = fmaxf(mx, __uint_as_float(s[b >> 1][(b & 1) * 16 + e]));
+                bm[b] = mx;
+            }
+            float rmax = bm[0];
+#pragma unroll
+            for (int b = 1; b < 8; ++b) rmax = fmaxf(rmax, bm[b]);
+            const float m_new = fmaxf(m, __fmul_rn(rmax, c2));
+            const float nm = -m_new;
+            const float alpha = ex2(__fsub_rn(m, m_new));
+            uint32_t scw0 = 0, scw1 = 0;
+            float rb[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const float a = ex2(__fsub_rn(__fmul_rn(bm[b], c2), m_new));
+                const uint32_t sc = cvt_e4m3(__fdiv_rn(a, 6.0f));
+                const float sv = e4m3_value(sc);
+                rb[b] = (sv == 0.0f) ? 0.0f : __frcp_rn(sv);
+                if (b < 4) scw0 |= sc << (8 * b);
+                else scw1 |= sc << (8 * (b - 4));
+            }
+            float sum = 0.0f;
+            uint32_t pc[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                const int b = h >> 1;
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float pe = ex2(fmaf(__uint_as_float(s[h >> 2][(h & 3) * 8 + e]), c2, nm));
+                    sum += pe;
+                    y[e] = pe * rb[b];
+                }
+                pc[h] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+            }
+            l = alpha * l + sum;
+
+            // P buffer and O are free once the previous P V has completed.
+            if (j > 0) {
+                if (!warp_wait(bars + kBarPvDone + i, (j - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            {
+                uint8_t *prow = P + (r >> 3) * 512 + (r & 7) * 64;
+                const int sw = (r & 7) >> 1;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16)
+                    *reinterpret_cast<uint4 *>(prow + ((c16 ^ sw) << 4)) =
+                        make_uint4(pc[4 * c16], pc[4 * c16 + 1], pc[4 * c16 + 2], pc[4 * c16 + 3]);
+                *reinterpret_cast<uint32_t *>(Psf + 16 * (r & 31) + 4 * (r >> 5)) = scw0;
+                *reinterpret_cast<uint32_t *>(Psf + 512 + 16 * (r & 31) + 4 * (r >> 5)) = scw1;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                // O = alpha * O for this warp's 32 rows
+                uint32_t o[D / 32][32];
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    reg_fence32(o[q]);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[q][e] = __float_as_uint(__uint_as_float(o[q][e]) * alpha);
+                    tmem_st32(trow + tO + 32 * q, o[q]);
+                }
+                tmem_st_wait();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bars + kBarPFull + i);
+            m = m_new;
+        }
+        if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
+            tc_fence_after();
+            const float inv = __frcp_rn(l);
+            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.N + grow) * D;
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t o[32];
+                tmem_ld32(trow + tO + 32 * q, o);
+                tmem_ld_wait();
+                reg_fence32(o);
+                if (grow < p.N) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                                        __uint_as_float(o[2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * q);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     cudaStream_t stream) {
+    using C = Cfg<D>;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int nqt = p.Np / kBlk;
+    const dim3 grid((nqt + 1) / 2, p.BH);
+    attn_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace attn
+
+inline cudaError_t launch_attn(const AttnParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                               const CUtensorMap &tm_v, int d, cudaStream_t stream) {
+    return d == 128 ? attn::launch_d<128>(p, tm_q, tm_k, tm_v, stream)
+                    : attn::launch_d<64>(p, tm_q, tm_k, tm_v, stream);
+}
+
+}  // namespace sa3

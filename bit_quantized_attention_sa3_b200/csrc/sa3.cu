@@ -1,0 +1,155 @@
+// sa3.cu -- libsa3: the C ABI declared in include/sa3.h.
+//
+// Single translation unit: the quantizer (quant.cuh) and attention kernel
+// (attn.cuh) are included here so that the device status word below is one
+// object without relocatable device code.  Host code validates arguments,
+// encodes the TMA tensor maps and enqueues the kernels on the caller's
+// stream; it allocates nothing.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sa3.h"
+#include "sa3_internal.h"
+#include "sm100.cuh"
+
+#include "attn.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D byte tensor [rows][inner] with a box of box_rows x box_inner bytes.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+              uint32_t box_rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1) return SA3_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SA3_ERR_UNSUPPORTED;
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    const int64_t Np = sa3_padded_len(N);
+    if (BH > 65535) return SA3_ERR_UNSUPPORTED;  // grid y
+    if (BH * Np * d / 2 >= (int64_t(1) << 31) || BH * Np >= (int64_t(1) << 31)) return SA3_ERR_UNSUPPORTED;
+    return SA3_OK;
+}
+
+int check_qkv(const sa3_qkv_fp4 *t) {
+    if (!t || !t->q_fp4 || !t->q_sf || !t->k_fp4 || !t->k_sf || !t->vt_fp4 || !t->vt_sf || !t->k_mean)
+        return SA3_ERR_INVALID_ARG;
+    if (!aligned16(t->q_fp4) || !aligned16(t->q_sf) || !aligned16(t->k_fp4) || !aligned16(t->k_sf) ||
+        !aligned16(t->vt_fp4) || !aligned16(t->vt_sf) || !aligned16(t->k_mean))
+        return SA3_ERR_INVALID_ARG;
+    return SA3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sa3_version(void) { return "libsa3 0.1.0 (sm_100a)"; }
+
+int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                     const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes, struct CUstream_st *stream) {
+    int rc = check_shape(B, H, N, d);
+    if (rc != SA3_OK) return rc;
+    if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
+    if ((rc = check_qkv(out)) != SA3_OK) return rc;
+    const int64_t need = sa3_quant_workspace_bytes(B, H, N, d);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
+    sa3::QuantParams p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.q_fp4 = static_cast<uint8_t *>(out->q_fp4);
+    p.q_sf = static_cast<uint8_t *>(out->q_sf);
+    p.k_fp4 = static_cast<uint8_t *>(out->k_fp4);
+    p.k_sf = static_cast<uint8_t *>(out->k_sf);
+    p.vt_fp4 = static_cast<uint8_t *>(out->vt_fp4);
+    p.vt_sf = static_cast<uint8_t *>(out->vt_sf);
+    p.k_mean = out->k_mean;
+    p.part = static_cast<double *>(workspace);
+    p.BH = B * H;
+    p.N = N;
+    p.Np = static_cast<int>(sa3_padded_len(N));
+    p.nchunk = (N + sa3::kQuantChunk - 1) / sa3::kQuantChunk;
+    return sa3::launch_quant(p, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK : SA3_ERR_CUDA;
+}
+
+int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,
+                 struct CUstream_st *stream) {
+    int rc = check_shape(B, H, N, d);
+    if (rc != SA3_OK) return rc;
+    if ((rc = check_qkv(in)) != SA3_OK) return rc;
+    if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
+    if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
+    const int BH = B * H;
+    const int Np = static_cast<int>(sa3_padded_len(N));
+    CUtensorMap tq, tk, tv;
+    const CUtensorMapSwizzle qk_sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    if (!make_map(&tq, in->q_fp4, d / 2, static_cast<uint64_t>(BH) * Np, d / 2, 128, qk_sw) ||
+        !make_map(&tk, in->k_fp4, d / 2, static_cast<uint64_t>(BH) * Np, d / 2, 128, qk_sw) ||
+        !make_map(&tv, in->vt_fp4, Np / 2, static_cast<uint64_t>(BH) * d, 64, d, CU_TENSOR_MAP_SWIZZLE_64B))
+        return SA3_ERR_CUDA;
+    sa3::AttnParams p;
+    p.q_sf = static_cast<const uint8_t *>(in->q_sf);
+    p.k_sf = static_cast<const uint8_t *>(in->k_sf);
+    p.vt_sf = static_cast<const uint8_t *>(in->vt_sf);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.BH = BH;
+    p.N = N;
+    p.Np = Np;
+    p.causal = causal;
+    p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+    return sa3::launch_attn(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA3_OK
+               : SA3_ERR_CUDA;
+}
+
+int sa3_device_status(struct CUstream_st *stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SA3_ERR_CUDA;
+    unsigned int st = 0;
+    if (cudaMemcpyFromSymbol(&st, sa3::g_sa3_status, sizeof(st)) != cudaSuccess) return SA3_ERR_CUDA;
+    if (st != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(sa3::g_sa3_status, &zero, sizeof(zero)) != cudaSuccess) return SA3_ERR_CUDA;
+        return SA3_ERR_TIMEOUT;
+    }
+    return SA3_OK;
+}
+
+}  // extern "C"

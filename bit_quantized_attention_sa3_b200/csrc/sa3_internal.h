@@ -1,0 +1,43 @@
+// sa3_internal.h -- launch parameters shared by the host API and kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace sa3 {
+
+constexpr int kQuantChunk = 512;  // tokens per fp64 partial sum of K
+
+struct QuantParams {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k;
+    const __nv_bfloat16 *v;
+    uint8_t *q_fp4;
+    uint8_t *q_sf;
+    uint8_t *k_fp4;
+    uint8_t *k_sf;
+    uint8_t *vt_fp4;
+    uint8_t *vt_sf;
+    float *k_mean;
+    double *part;  // [BH][nchunk][d] scratch
+    int BH;
+    int N;
+    int Np;
+    int nchunk;
+};
+
+struct AttnParams {
+    const uint8_t *q_sf;
+    const uint8_t *k_sf;
+    const uint8_t *vt_sf;
+    __nv_bfloat16 *out;
+    int BH;
+    int N;
+    int Np;
+    int causal;
+    float scale_log2;  // fp32(sm_scale * log2 e)
+};
+
+}  // namespace sa3

@@ -1,0 +1,169 @@
+/*
+ * sa3.h -- C ABI of libsa3: microscaled-FP4 attention forward on B200
+ * (sm_100a).
+ *
+ * The method ("SageAttention3: Microscaling FP4 Attention for Inference and
+ * An Exploration of 8-Bit Training", abstract) computes attention on the
+ * Blackwell FP4 tensor cores: K is first smoothed by subtracting its mean
+ * over tokens, which leaves softmax attention unchanged ("SageAttention:
+ * Accurate 8-Bit Attention for Plug-and-play Inference Acceleration",
+ * section "Approach"); Q, K and V are quantized to FP4 E2M1 with one E4M3
+ * scale per 16 elements; S = Q K^T and O = P V run as block-scaled FP4
+ * matrix products, with P quantized the same way once per 128-token KV
+ * block against the running row maximum of a blockwise online softmax.
+ *
+ * Conventions for every call:
+ *   - every pointer argument is a DEVICE pointer (cudaMalloc'ed or from a
+ *     caching allocator) unless stated otherwise; the library never
+ *     allocates, frees or keeps a reference to caller memory;
+ *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream); a return of SA3_OK means the arguments were valid
+ *     and the kernels were enqueued, not that they have finished;
+ *   - shapes: B, H >= 1; N >= 1; d in {64, 128}; B*H*N_p*d/2 < 2^31
+ *     where N_p = N rounded up to a multiple of 128;
+ *   - Q, K, V and the output are bf16, contiguous [B][H][N][d], 16-byte
+ *     aligned;
+ *   - the library is thread-safe for concurrent calls on different streams
+ *     as long as their workspaces differ.
+ *
+ * Error behaviour: arguments are checked before any launch; a bad argument
+ * returns SA3_ERR_INVALID_ARG (null pointer, misalignment, non-positive
+ * size, workspace too small) or SA3_ERR_UNSUPPORTED (d not 64/128, size
+ * limits) and enqueues nothing.  A failed launch returns SA3_ERR_CUDA.
+ * Device-side waits are bounded; if one gives up, the kernel records
+ * SA3_ERR_TIMEOUT in a device status word, releases what it holds and
+ * returns; sa3_device_status() reports it.
+ */
+#ifndef SA3_H
+#define SA3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t */
+
+typedef enum {
+    SA3_OK = 0,
+    SA3_ERR_INVALID_ARG = 1,
+    SA3_ERR_UNSUPPORTED = 2,
+    SA3_ERR_CUDA = 3,
+    SA3_ERR_TIMEOUT = 4
+} sa3_status;
+
+/*
+ * Quantized operands produced by sa3_quantize_qkv and consumed by
+ * sa3_attn_fwd.  All device pointers, caller-owned, sizes from the helpers
+ * below.  Layouts (bh = b*H + h, N_p = sa3_padded_len(N)):
+ *
+ *   q_fp4, k_fp4  u8 [B*H][N_p][d/2]: E2M1 codes, row-major, element 2i in
+ *                 the low nibble of byte i, element 2i+1 in the high one.
+ *   vt_fp4        u8 [B*H][d][N_p/2]: V transposed (channel-major), same
+ *                 packing along tokens.
+ *   q_sf, k_sf    E4M3 scale of the 16 elements (t, 16c .. 16c+15) stored at
+ *                   (((bh*(N_p/128) + t/128)*(d/64) + c/4) * 512
+ *                    + 16*(t%32) + 4*((t%128)/32) + c%4
+ *                 i.e. 512-byte atoms of 128 tokens x 4 scales in the order
+ *                 the tensor core's block-scaled MMA reads them.
+ *   vt_sf         E4M3 scale of the 16 tokens (16u .. 16u+15) of channel c:
+ *                   (bh*(N_p/64) + u/4) * 512 + 16*(c%32) + 4*(c/32) + u%4
+ *                 (channels padded to 128; padding channels hold 0).
+ *   k_mean        fp32 [B*H][d]: the mean of K over its N tokens.
+ *
+ * Tokens t >= N have code 0 and scale 0.  A block whose scale rounds to 0
+ * has all codes 0.
+ */
+typedef struct sa3_qkv_fp4 {
+    void *q_fp4;
+    void *q_sf;
+    void *k_fp4;
+    void *k_sf;
+    void *vt_fp4;
+    void *vt_sf;
+    float *k_mean;
+} sa3_qkv_fp4;
+
+/* ---- sizes (bytes); header-only helpers, not exported ---------------- */
+static inline int64_t sa3_padded_len(int64_t N) { return (N + 127) / 128 * 128; }
+static inline int64_t sa3_qk_fp4_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ return B * H * sa3_padded_len(N) * d / 2; }
+static inline int64_t sa3_qk_sf_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ return B * H * sa3_padded_len(N) * d / 16; }
+static inline int64_t sa3_vt_fp4_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ return B * H * d * sa3_padded_len(N) / 2; }
+static inline int64_t sa3_vt_sf_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ (void)d; return B * H * sa3_padded_len(N) * 8; }
+static inline int64_t sa3_kmean_bytes(int64_t B, int64_t H, int64_t d) { return B * H * d * 4; }
+/* Scratch for the K-mean reduction: fp64 partial sums per 512 tokens. */
+static inline int64_t sa3_quant_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ return B * H * ((N + 511) / 512) * d * 8; }
+
+/*
+ * sa3_quantize_qkv -- K smoothing plus FP4 microscaling of Q, K and V.
+ *
+ * Steps ("SageAttention" summary, "Approach"; "SageAttention3" abstract):
+ *   mean[bh][c] = fp32( (sum_t K[bh][t][c] in fp64) / N in fp64 )
+ *   K_s = fp32(K) - mean            (one fp32 subtraction; K is not modified)
+ *   for every 16-element block x of Q, K_s (along d) and V (along tokens):
+ *     s = E4M3_RN_satfinite(fp32(max|x| / 6)), r = fp32(1/s),
+ *     code_i = E2M1_RN_satfinite(fp32(x_i * r)), all codes 0 if s == 0.
+ * Rounding is to nearest even; a negative value that rounds to zero keeps
+ * its sign (code 0x8).  The fp64 sums are bit-identical to any other
+ * order whenever they are exact, which holds for bf16 inputs whose
+ * magnitudes span less than 2^30 at N <= 2^15.
+ *
+ * q, k, v    : bf16 [B][H][N][d], device, 16-byte aligned, read only.
+ * out        : the seven output buffers above (device; written).
+ * workspace  : device scratch of at least sa3_quant_workspace_bytes bytes
+ *              (contents on entry are ignored).
+ * Returns SA3_OK or an error code (see top of file).
+ */
+int sa3_quantize_qkv(const void *q, const void *k, const void *v,
+                     int B, int H, int N, int d,
+                     const sa3_qkv_fp4 *out,
+                     void *workspace, size_t workspace_bytes,
+                     struct CUstream_st *stream);
+
+/*
+ * sa3_attn_fwd -- O = softmax(Q^ K^T * sm_scale) V^ with FP4 P, bf16 out.
+ *
+ * Per (bh, 128-row Q block), for KV blocks j = 0.. (causal: j <= Q block):
+ *   S = Q^ K^_j^T on the block-scaled FP4 tensor cores (fp32 accumulate);
+ *   t = S * fp32(sm_scale * log2 e); columns >= N and, if causal, columns
+ *   > row are -inf; m' = max(m, rowmax t); alpha = 2^(m - m');
+ *   P = 2^(t - m'); l = alpha*l + rowsum(P);
+ *   P^ = P microscaled per 16 columns exactly as in sa3_quantize_qkv;
+ *   O = alpha*O + P^ V^_j (block-scaled FP4, fp32 accumulate); m = m'.
+ * out = bf16_RN(O / l).  ("Online normalizer calculation for softmax" and
+ * the FlashAttention papers, in the SageAttention3 reference list.)
+ *
+ * in       : quantized operands from sa3_quantize_qkv for the same shape.
+ * causal   : 0 or 1 (mask col > row, rows and columns both from 0).
+ * sm_scale : softmax scale; <= 0 selects 1/sqrt(d).
+ * out      : bf16 [B][H][N][d], device, 16-byte aligned (written).
+ * Returns SA3_OK or an error code (see top of file).
+ */
+int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d,
+                 int causal, float sm_scale, void *out,
+                 struct CUstream_st *stream);
+
+/*
+ * sa3_device_status -- synchronizes `stream`, returns SA3_ERR_TIMEOUT if
+ * a kernel of this library gave up on a bounded wait since the last call
+ * (and clears the record), SA3_ERR_CUDA if the stream reports an error,
+ * else SA3_OK.
+ */
+int sa3_device_status(struct CUstream_st *stream);
+
+/* Library version string, e.g. "libsa3 0.1.0 (sm_100a)". Host memory,
+ * static, never freed. */
+const char *sa3_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA3_H */

@@ -1,0 +1,56 @@
+"""The C ABI without a GPU: libsa3.so loads, exports every function that
+include/sa3.h declares, returns its version, and rejects bad arguments
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sa3.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|char|void)\s*\*?\s*(sa3_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_quantized_attention_sa3_b200 import build
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def test_header_declares_the_boundary():
+    assert _declared() == ["sa3_attn_fwd", "sa3_device_status", "sa3_quantize_qkv", "sa3_version"]
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_version(lib):
+    lib.sa3_version.restype = ctypes.c_char_p
+    assert lib.sa3_version().decode().startswith("libsa3")
+
+
+def test_argument_checks_need_no_gpu(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.sa3_quantize_qkv.restype = I
+    lib.sa3_quantize_qkv.argtypes = [P, P, P, I, I, I, I, P, P, ctypes.c_size_t, P]
+    lib.sa3_attn_fwd.restype = I
+    lib.sa3_attn_fwd.argtypes = [P, I, I, I, I, I, ctypes.c_float, P, P]
+    # d unsupported
+    assert lib.sa3_quantize_qkv(16, 16, 16, 1, 1, 8, 96, None, None, 0, None) == 2
+    # null pointers / bad sizes
+    assert lib.sa3_quantize_qkv(None, None, None, 1, 1, 8, 64, None, None, 0, None) == 1
+    assert lib.sa3_quantize_qkv(16, 16, 16, 0, 1, 8, 64, None, None, 0, None) == 1
+    assert lib.sa3_attn_fwd(None, 1, 1, 8, 64, 0, 0.0, None, None) == 1
+    assert lib.sa3_attn_fwd(None, 1, 1, 8, 100, 0, 0.0, None, None) == 2
+    # B*H beyond the grid limit
+    assert lib.sa3_attn_fwd(None, 1000, 1000, 8, 64, 0, 0.0, None, None) == 2

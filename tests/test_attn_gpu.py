@@ -1,0 +1,135 @@
+"""sa3_attn_fwd on the GPU against the CPU oracle.
+
+Bar: output rel-L2 <= 2e-3 against the oracle on the same quantized
+operands (the GPU takes its exponentials with ex2.approx and accumulates in
+the tensor core, so P codes may flip at rounding boundaries; the oracle
+uses exp2f and fp64 sums).  The GPU is also checked against fp64 exact
+attention of the bf16 inputs: its cosine must be within 1e-3 of the
+oracle's own cosine (the method's accuracy, not a kernel property).
+
+Small shapes are compared in full; the benchmark workloads at full size
+are compared on sampled Q blocks (block 0, the last block with its ragged
+tail or longest causal rows, and two seeded random blocks per (b, h))."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sa3_inputs
+from sa3_testutil import bits_to_f32, cosine, qk_sf_to_canonical, rel_l2, sample_units, vt_sf_to_canonical
+
+sa3 = pytest.importorskip("bit_quantized_attention_sa3_b200")
+
+TOL = 2e-3
+
+
+def _canonical(qz, B, H, N, d):
+    Np = sa3.padded_len(N)
+    return dict(q_codes=qz.q_fp4.cpu().numpy(), k_codes=qz.k_fp4.cpu().numpy(),
+                vt_codes=qz.vt_fp4.cpu().numpy(),
+                q_sf=qk_sf_to_canonical(qz.q_sf.cpu().numpy(), B, H, Np, d),
+                k_sf=qk_sf_to_canonical(qz.k_sf.cpu().numpy(), B, H, Np, d),
+                vt_sf=vt_sf_to_canonical(qz.vt_sf.cpu().numpy(), B, H, Np, d))
+
+
+def _run(name, over, causal, units=None):
+    q, k, v = sa3_inputs.make_qkv(name, shape_override=over)
+    B, H, N, d = q.shape
+    qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
+    out = sa3.attn_fwd(qz, causal=causal)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    canon = _canonical(qz, B, H, N, d)
+    ref = bits_to_f32(oracle.attn_fwd(canon, N, causal, units=units))
+    ex = oracle.attn_exact(q, k, v, causal, units=units)
+    if units is None:
+        mask = np.ones((B * H, N), bool)
+    else:
+        mask = np.zeros((B * H, N), bool)
+        for bh, qb in units:
+            mask[bh, qb * 128: min(N, qb * 128 + 128)] = True
+    g = got.reshape(B * H, N, d)[mask]
+    r = ref.reshape(B * H, N, d)[mask]
+    e = ex.reshape(B * H, N, d)[mask]
+    return rel_l2(g, r), cosine(g, e), cosine(r, e)
+
+
+SMALL = [
+    ("tiny_b1h2n256d64", None),
+    ("tiny_b1h2n256d64", {"N": 1}),
+    ("tiny_b1h2n256d64", {"N": 15}),
+    ("tiny_b1h2n256d64", {"N": 129}),
+    ("tiny_b1h2n256d64", {"N": 300, "H": 3}),
+    ("tiny_b1h2n256d64", {"N": 640}),
+    ("noncausal_b2h16n4096d128", {"B": 1, "H": 2, "N": 16}),
+    ("noncausal_b2h16n4096d128", {"B": 1, "H": 2, "N": 127}),
+    ("noncausal_b2h16n4096d128", {"B": 2, "H": 2, "N": 640}),
+    ("noncausal_b2h16n4096d128", {"B": 1, "H": 3, "N": 1000}),
+]
+
+
+def _ids(c):
+    return c[0] + ("" if c[1] is None else "-" + "-".join(f"{k}{v}" for k, v in c[1].items()))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["noncausal", "causal"])
+@pytest.mark.parametrize("case", SMALL, ids=[_ids(c) for c in SMALL])
+def test_attn_matches_oracle_small(case, causal):
+    err, cos_gpu, cos_oracle = _run(case[0], case[1], causal)
+    assert err <= TOL, f"rel-L2 vs oracle {err:.3e}"
+    assert cos_gpu >= cos_oracle - 1e-3
+
+
+FULL = [
+    ("noncausal_b2h16n4096d128", False),
+    ("videodit_b1h30n17776d64", False),
+    ("prefill_b4h32n8192d128_causal", True),
+    ("longctx_b1h32n32768d128_causal", True),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", FULL, ids=[c[0] for c in FULL])
+def test_attn_matches_oracle_full_size_sampled(case):
+    name, causal = case
+    w = sa3_inputs.WORKLOADS[name]
+    bh_list = None
+    if w.B * w.H > 32:
+        rng = np.random.default_rng(2)
+        bh_list = sorted({0, w.B * w.H - 1} | set(int(x) for x in rng.choice(w.B * w.H, 14, replace=False)))
+    units = sample_units(w.B, w.H, w.N, seed=3, per_bh=2, bh_list=bh_list)
+    err, cos_gpu, cos_oracle = _run(name, None, causal, units=units)
+    print(f"{name}: rel-L2 vs oracle {err:.3e}, cosine vs exact gpu {cos_gpu:.5f} oracle {cos_oracle:.5f}")
+    assert err <= TOL
+    assert cos_gpu >= cos_oracle - 1e-3
+
+
+@pytest.mark.gpu
+def test_attn_sm_scale_and_repeatability():
+    q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 384})]
+    B, H, N, d = q.shape
+    qz = sa3.quantize_qkv(q, k, v)
+    a = sa3.attn_fwd(qz, causal=False, sm_scale=0.05)
+    b = sa3.attn_fwd(qz, causal=False, sm_scale=0.05)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    canon = _canonical(qz, B, H, N, d)
+    ref = bits_to_f32(oracle.attn_fwd(canon, N, False, sm_scale=0.05))
+    assert rel_l2(a.float().cpu().numpy(), ref) <= TOL
+
+
+@pytest.mark.gpu
+def test_attn_rejects_bad_arguments():
+    q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64")]
+    qz = sa3.quantize_qkv(q, k, v)
+    bad = sa3.QuantizedQKV(**{**qz.__dict__, "d": 80})
+    with pytest.raises(sa3.Sa3Error) as e:
+        sa3.attn_fwd(bad)
+    assert e.value.code == sa3.SA3_ERR_UNSUPPORTED
+    mis = torch.empty(q.numel() + 8, dtype=torch.bfloat16, device="cuda")[1:1 + q.numel()].view(q.shape)
+    with pytest.raises(sa3.Sa3Error) as e:
+        sa3.attn_fwd(qz, out=mis)
+    assert e.value.code == sa3.SA3_ERR_INVALID_ARG
