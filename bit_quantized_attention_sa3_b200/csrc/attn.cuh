@@ -68,7 +68,8 @@ struct Cfg {
     static constexpr int oP1 = oP0 + kPBytes;
     static constexpr int oPsf0 = oP1 + kPBytes;
     static constexpr int oPsf1 = oPsf0 + kPsfBytes;
-    static constexpr int oBar = oPsf1 + kPsfBytes;
+    static constexpr int oLut = oPsf1 + kPsfBytes;     // 256 floats: 1 / E4M3 value
+    static constexpr int oBar = oLut + 1024;
     static constexpr int kSmemBytes = oBar + 256 + 1024;
     // TMEM columns
     static constexpr uint32_t tS = 0;
@@ -100,6 +101,51 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+constexpr float kSixth = 1.0f / 6.0f;
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// Packed fp32 pairs (low word = first element) and the sm_100 f32x2 ops.
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float lo2(uint64_t v) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+    return a;
+}
+__device__ __forceinline__ float hi2(uint64_t v) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+    return b;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// E4M3 codes of two floats: byte 0 from `lo`, byte 1 from `hi`.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+    return out;
 }
 
 // mbar_wait with a warp-uniform result, for code that continues with
@@ -165,6 +211,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (threadIdx.x < 256) {
+        // exact IEEE reciprocal of every E4M3 scale; 0 for scale 0 (and NaN codes)
+        const float v = e4m3_value(threadIdx.x);
+        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] =
+            (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
+    }
     if (warp == 9) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
@@ -173,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const float *rcp_lut = reinterpret_cast<const float *>(base + C::oLut);
 
     if (warp >= 8) {
       if (warp == 8) {
@@ -341,45 +394,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (32 * q + e >= lim) s[q][e] = __float_as_uint(-INFINITY);
                 }
             }
+            // block maxima of the raw scores (c > 0, so max commutes with * c)
             float bm[8];
 #pragma unroll
             for (int b = 0; b < 8; ++b) {
-                float mx = __uint_as_float(s[b >> 1][(b & 1) * 16]);
-#pragma unroll
-                for (int e = 1; e < 16; ++e) mx = fmaxf(mx, __uint_as_float(s[b >> 1][(b & 1) * 16 + e]));
-                bm[b] = mx;
+                const uint32_t *x = &s[b >> 1][(b & 1) * 16];
+                const float m0 = max3f(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]));
+                const float m1 = max3f(__uint_as_float(x[3]), __uint_as_float(x[4]), __uint_as_float(x[5]));
+                const float m2 = max3f(__uint_as_float(x[6]), __uint_as_float(x[7]), __uint_as_float(x[8]));
+                const float m3 = max3f(__uint_as_float(x[9]), __uint_as_float(x[10]), __uint_as_float(x[11]));
+                const float m4 = max3f(__uint_as_float(x[12]), __uint_as_float(x[13]), __uint_as_float(x[14]));
+                bm[b] = max3f(max3f(m0, m1, m2), max3f(m3, m4, __uint_as_float(x[15])), m0);
             }
-            float rmax = bm[0];
-#pragma unroll
-            for (int b = 1; b < 8; ++b) rmax = fmaxf(rmax, bm[b]);
+            const float rmax = max3f(max3f(bm[0], bm[1], bm[2]), max3f(bm[3], bm[4], bm[5]), fmaxf(bm[6], bm[7]));
             const float m_new = fmaxf(m, __fmul_rn(rmax, c2));
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
-            uint32_t scw0 = 0, scw1 = 0;
+            // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
+            // two blocks per conversion; r_b = 1/s_b from the exact table
+            uint32_t scw[2];
             float rb[8];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const float a = ex2(__fsub_rn(__fmul_rn(bm[b], c2), m_new));
-                const uint32_t sc = cvt_e4m3(__fdiv_rn(a, 6.0f));
-                const float sv = e4m3_value(sc);
-                rb[b] = (sv == 0.0f) ? 0.0f : __frcp_rn(sv);
-                if (b < 4) scw0 |= sc << (8 * b);
-                else scw1 |= sc << (8 * (b - 4));
+            for (int b = 0; b < 8; b += 2) {
+                const float a0 = ex2(__fsub_rn(__fmul_rn(bm[b], c2), m_new));
+                const float a1 = ex2(__fsub_rn(__fmul_rn(bm[b + 1], c2), m_new));
+                const uint32_t sc2 = cvt_e4m3x2(a1 * kSixth, a0 * kSixth);  // byte 0: block b
+                rb[b] = rcp_lut[sc2 & 0xFF];
+                rb[b + 1] = rcp_lut[sc2 >> 8];
+                if ((b & 2) == 0) scw[b >> 2] = sc2;
+                else scw[b >> 2] |= sc2 << 16;
             }
-            float sum = 0.0f;
+            // P = 2^(t - m'), row sum of P (tree per block), codes of P * r
+            const uint64_t cc = pack2(c2, c2);
+            const uint64_t nn = pack2(nm, nm);
+            uint64_t acc = pack2(0.0f, 0.0f);
             uint32_t pc[16];
 #pragma unroll
-            for (int h = 0; h < 16; ++h) {
-                const int b = h >> 1;
-                float y[8];
+            for (int b = 0; b < 8; ++b) {
+                const uint32_t *x = &s[b >> 1][(b & 1) * 16];
+                uint64_t vp[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float pe = ex2(fmaf(__uint_as_float(s[h >> 2][(h & 3) * 8 + e]), c2, nm));
-                    sum += pe;
-                    y[e] = pe * rb[b];
+                for (int i = 0; i < 8; ++i) {
+                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), cc, nn);
+                    vp[i] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
                 }
-                pc[h] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+                const uint64_t s01 = add2(add2(vp[0], vp[1]), add2(vp[2], vp[3]));
+                const uint64_t s23 = add2(add2(vp[4], vp[5]), add2(vp[6], vp[7]));
+                acc = add2(acc, add2(s01, s23));
+                const uint64_t rr = pack2(rb[b], rb[b]);
+                uint64_t vy[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) vy[i] = mul2(vp[i], rr);
+                pc[2 * b] = cvt_e2m1x8(lo2(vy[0]), hi2(vy[0]), lo2(vy[1]), hi2(vy[1]), lo2(vy[2]), hi2(vy[2]),
+                                       lo2(vy[3]), hi2(vy[3]));
+                pc[2 * b + 1] = cvt_e2m1x8(lo2(vy[4]), hi2(vy[4]), lo2(vy[5]), hi2(vy[5]), lo2(vy[6]), hi2(vy[6]),
+                                           lo2(vy[7]), hi2(vy[7]));
             }
+            const float sum = lo2(acc) + hi2(acc);
+            const uint32_t scw0 = scw[0], scw1 = scw[1];
             l = alpha * l + sum;
 
             // P buffer and O are free once the previous P V has completed.
@@ -407,10 +479,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < D / 32; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
                 tmem_ld_wait();
 #pragma unroll
+                const uint64_t aa = pack2(alpha, alpha);
+#pragma unroll
                 for (int q = 0; q < D / 32; ++q) {
                     reg_fence32(o[q]);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[q][e] = __float_as_uint(__uint_as_float(o[q][e]) * alpha);
+                    for (int e = 0; e < 32; e += 2) {
+                        const uint64_t v = mul2(pack2(__uint_as_float(o[q][e]), __uint_as_float(o[q][e + 1])), aa);
+                        o[q][e] = __float_as_uint(lo2(v));
+                        o[q][e + 1] = __float_as_uint(hi2(v));
+                    }
                     tmem_st32(trow + tO + 32 * q, o[q]);
                 }
                 tmem_st_wait();
