@@ -75,6 +75,27 @@ int check_qkv(const sa3_qkv_fp4 *t) {
     return SA3_OK;
 }
 
+// Scratch for sa3_quantize_qkv_noalloc: one fixed array per device that
+// loads the library (fp64 K-mean partial sums).
+static __device__ __align__(256) double g_noalloc_scratch[SA3_NOALLOC_SCRATCH_BYTES / sizeof(double)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of this device's scratch array, looked up once per device
+// with that device current (host code must not pass the symbol itself).
+void *noalloc_scratch(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -106,6 +127,21 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, 
     p.Np = static_cast<int>(sa3_padded_len(N));
     p.nchunk = (N + sa3::kQuantChunk - 1) / sa3::kQuantChunk;
     return sa3::launch_quant(p, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK : SA3_ERR_CUDA;
+}
+
+int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                             const sa3_qkv_fp4 *out, struct CUstream_st *stream) {
+    int rc = check_shape(B, H, N, d);
+    if (rc != SA3_OK) return rc;
+    if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
+    if ((rc = check_qkv(out)) != SA3_OK) return rc;
+    if (sa3_quant_workspace_bytes(B, H, N, d) > static_cast<int64_t>(SA3_NOALLOC_SCRATCH_BYTES))
+        return SA3_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA3_ERR_CUDA;
+    void *scratch = noalloc_scratch(dev);
+    if (!scratch) return SA3_ERR_CUDA;
+    return sa3_quantize_qkv(q, k, v, B, H, N, d, out, scratch, SA3_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,

@@ -151,6 +151,37 @@ int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d,
                  struct CUstream_st *stream);
 
 /*
+ * sa3_quantize_qkv_noalloc -- sa3_quantize_qkv without a caller workspace.
+ *
+ * There is no counterpart in the paper: this is a convenience for callers
+ * that cannot hand the library device memory at call time, for instance a
+ * plug-in layer inside a framework that owns every device allocation and
+ * exposes no allocator to plug-ins, or a latency-critical path where a
+ * cudaMalloc (which may synchronize the device) is not acceptable.
+ *
+ * Same arguments, outputs and results as sa3_quantize_qkv, minus the
+ * workspace: the K-mean partial sums go to a fixed scratch array that the
+ * library holds in device memory on every GPU that loads it, until the
+ * process exits.  The array holds SA3_NOALLOC_SCRATCH_BYTES bytes, so the
+ * call accepts shapes with sa3_quant_workspace_bytes(B, H, N, d) <=
+ * SA3_NOALLOC_SCRATCH_BYTES and returns SA3_ERR_UNSUPPORTED otherwise.
+ * It calls no allocation routine.
+ *
+ * The first call on a device looks up that device's copy of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call
+ * outside any stream capture.  All calls share the one array: two calls
+ * whose kernels overlap on the GPU (different streams without ordering)
+ * race on it and give undefined results.  Nothing in the array needs to
+ * start at zero -- every call rewrites all the scratch it reads -- and it
+ * keeps the last call's contents.
+ */
+#define SA3_NOALLOC_SCRATCH_BYTES (4u << 20)
+int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v,
+                             int B, int H, int N, int d,
+                             const sa3_qkv_fp4 *out,
+                             struct CUstream_st *stream);
+
+/*
  * sa3_device_status -- synchronizes `stream`, returns SA3_ERR_TIMEOUT if
  * a kernel of this library gave up on a bounded wait since the last call
  * (and clears the record), SA3_ERR_CUDA if the stream reports an error,

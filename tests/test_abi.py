@@ -26,7 +26,8 @@ def lib():
 
 
 def test_header_declares_the_boundary():
-    assert _declared() == ["sa3_attn_fwd", "sa3_device_status", "sa3_quantize_qkv", "sa3_version"]
+    assert _declared() == ["sa3_attn_fwd", "sa3_device_status", "sa3_quantize_qkv",
+                           "sa3_quantize_qkv_noalloc", "sa3_version"]
 
 
 def test_library_exports_every_declared_symbol(lib):
