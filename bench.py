@@ -144,6 +144,25 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, 2 ms"}
 
 
+def profiled_traffic(kernel_src: str, profile: str):
+    """DRAM bytes per launch recorded in a committed ncu summary, or None if
+    the kernel source has changed since (sha256 prefix recorded there)."""
+    import hashlib
+    try:
+        src = open(os.path.join(ROOT, kernel_src), "rb").read()
+        txt = open(os.path.join(ROOT, "profiles", profile)).read()
+    except OSError:
+        return None
+    sha = hashlib.sha256(src).hexdigest()[:16]
+    rec = dict(line.split(": ", 1) for line in txt.splitlines() if line.startswith(("source_sha256_16: ",)))
+    if rec.get("source_sha256_16", "").strip() != sha:
+        return None
+    for line in txt.splitlines():
+        if line.startswith("| dram_bytes_per_launch |"):
+            return int(line.split("|")[2].strip())
+    return None
+
+
 def run_sa3(args, rank, world, local):
     import bit_quantized_attention_sa3_b200 as sa3
     torch.cuda.set_device(local)
@@ -257,7 +276,9 @@ def run_sa3(args, rank, world, local):
         "quantize": {"ms": round(t_quant, 4), "GB_per_s": round(qk_bytes / (t_quant * 1e-3) / 1e9, 1),
                      "algorithmic_bytes": qk_bytes},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                     "traffic": profiled_traffic("bit_quantized_attention_sa3_b200/csrc/attn.cuh",
+                                                 "attn_fwd_kernel_d128_noncausal_b2h16n4096d128.md"),
                      "kernel": "attn_fwd_kernel<128>",
                      "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"},
         "e2e": {"value": round(world * ops / (t_e2e * 1e-3) / 1e12, 2), "unit": UNIT, "ms": round(t_e2e, 4),

@@ -10,25 +10,21 @@
 //   O = alpha*O + P^ V^_j              block-scaled FP4 MMA, fp32 in TMEM
 // and finally out = bf16(O / l).
 //
-// One CTA = two 128-row Q tiles of one (b, h), 16 warps:
-//   warps 0-3   softmax for Q tile 0 (one thread per row = one TMEM lane)
-//   warps 4-7   softmax for Q tile 1
-//   warp  8     producer: TMA loads of Q, and of K / V^T codes + scales into
-//               a 3-stage ring (mbarrier transaction counts)
-//   warp  9     allocates TMEM and issues every tcgen05 op from one thread:
-//               scale-factor copies (tcgen05.cp), S = Q K^T, O += P V
-//   warps 12-15 rescale O in TMEM (O *= alpha) between consecutive P V
-//               products and write the bf16 output; the softmax groups hand
-//               them alpha as soon as the row maximum is known, so the
-//               TMEM round trip overlaps the exponentials
+// One CTA = two 128-row Q tiles of one (b, h), 12 warps:
+//   warps 0-3  softmax for Q tile 0 (one thread per row = one TMEM lane)
+//   warps 4-7  softmax for Q tile 1
+//   warp  8    producer: TMA loads of Q, and of K / V^T codes + scales into
+//              a 3-stage ring (mbarrier transaction counts)
+//   warp  9    allocates TMEM and issues every tcgen05 op from one thread:
+//              scale-factor copies (tcgen05.cp), S = Q K^T, O += P V
+//   warps 10-11 idle (registers are granted per warpgroup)
 // TMEM (512 columns): S (128, shared by both tiles -- each softmax group
 // loads it to registers at once and releases it), O0, O1 (d each), and
 // the scale factors of Q0, Q1, K, P and V.  tcgen05.cp and tcgen05.mma
 // from one thread execute in issue order, so each scale-factor region is
 // rewritten right before the MMA that reads it.  P goes through shared
-// memory (64-byte swizzled K-major rows + 512-byte scale atoms, double
-// buffered by KV block parity) because the block-scaled FP4 MMA takes A
-// from shared memory only.
+// memory (64-byte swizzled K-major rows + 512-byte scale atoms) because
+// the block-scaled FP4 MMA takes A from shared memory only.
 // The tensor pipe order per KV block j is QK0(j+1), PV0(j), QK1(j+1),
 // PV1(j): each softmax group finds its next S ready as soon as it has
 // produced its P, so the two groups run concurrently and the exp / FMA
@@ -43,15 +39,7 @@ namespace attn {
 
 constexpr int kBlk = 128;
 constexpr int kStages = 3;
-constexpr int kThreads = 512;  // four warpgroups
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
-constexpr int kWarpCorr = 12;   // warps 12-15: O correction and epilogue
-// Register split (setmaxnreg) of the 512 x 128 launch allocation: softmax
-// 168, producer/MMA 80, correction 96: 256*168 + 128*80 + 128*96 = 65536.
-constexpr int kRegsSoftmax = 168;
-constexpr int kRegsLoad = 80;
-constexpr int kRegsCorr = 96;
+constexpr int kThreads = 384;  // three warpgroups, 168 registers per thread
 
 template <int D>
 struct Cfg {
@@ -76,15 +64,13 @@ struct Cfg {
     static constexpr int sKsf = sV + al(kVBytes);
     static constexpr int sVsf = sKsf + kSfBytes;
     static constexpr int kStageBytes = al(sVsf + kVsfBytes);
-    // P of tile i, buffer u (= KV block parity): codes at oP + (2i+u)*kPBytes,
-    // scale atoms at oPsf + (2i+u)*kPsfBytes
-    static constexpr int oP = oStage + kStages * kStageBytes;
-    static constexpr int oPsf = oP + 4 * kPBytes;
-    static constexpr int oLut = oPsf + 4 * kPsfBytes;  // 256 floats: 1 / E4M3 value
-    static constexpr int oAlpha = oLut + 1024;         // [tile][parity][128] floats
-    static constexpr int oL = oAlpha + 2048;           // [tile][128] floats
-    static constexpr int oBar = oL + 1024;
-    static constexpr int kSmemBytes = oBar + 512 + 1024;
+    static constexpr int oP0 = oStage + kStages * kStageBytes;
+    static constexpr int oP1 = oP0 + kPBytes;
+    static constexpr int oPsf0 = oP1 + kPBytes;
+    static constexpr int oPsf1 = oPsf0 + kPsfBytes;
+    static constexpr int oLut = oPsf1 + kPsfBytes;     // 256 floats: 1 / E4M3 value
+    static constexpr int oBar = oLut + 1024;
+    static constexpr int kSmemBytes = oBar + 256 + 1024;
     // TMEM columns
     static constexpr uint32_t tS = 0;
     static constexpr uint32_t tO0 = 128;
@@ -103,15 +89,12 @@ enum : int {
     kBarQ = 0,
     kBarKvFull = 1,                  // kStages
     kBarKvEmpty = 1 + kStages,       // kStages
-    kBarSFull = 1 + 2 * kStages,     // 2: [tile]
+    kBarSFull = 1 + 2 * kStages,     // 2
     kBarSEmpty = 3 + 2 * kStages,    // 1
-    kBarPFull = 4 + 2 * kStages,     // 4: [tile][parity]
-    kBarPvDone = 8 + 2 * kStages,    // 4: [tile][parity]
-    kBarAlpha = 12 + 2 * kStages,    // 4: [tile][parity]
-    kBarCorr = 16 + 2 * kStages,     // 2: [tile]
-    kBarL = 18 + 2 * kStages,        // 2: [tile]
-    kBarDrain = 20 + 2 * kStages,    // 1
-    kBarCount = 21 + 2 * kStages
+    kBarPFull = 4 + 2 * kStages,     // 2
+    kBarPvDone = 6 + 2 * kStages,    // 2
+    kBarDrain = 8 + 2 * kStages,     // 1
+    kBarCount = 9 + 2 * kStages
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -217,17 +200,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bars + kBarKvFull + s, 1);
             mbar_init(bars + kBarKvEmpty + s, 1);
         }
+        mbar_init(bars + kBarSFull + 0, 1);
+        mbar_init(bars + kBarSFull + 1, 1);
         mbar_init(bars + kBarSEmpty, 128);
-        for (int x = 0; x < 2; ++x) {
-            mbar_init(bars + kBarSFull + x, 1);
-            mbar_init(bars + kBarCorr + x, 128);
-            mbar_init(bars + kBarL + x, 128);
-        }
-        for (int x = 0; x < 4; ++x) {
-            mbar_init(bars + kBarPFull + x, 128);
-            mbar_init(bars + kBarPvDone + x, 1);
-            mbar_init(bars + kBarAlpha + x, 128);
-        }
+        mbar_init(bars + kBarPFull + 0, 128);
+        mbar_init(bars + kBarPFull + 1, 128);
+        mbar_init(bars + kBarPvDone + 0, 1);
+        mbar_init(bars + kBarPvDone + 1, 1);
         mbar_init(bars + kBarDrain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -235,9 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x < 256) {
         // exact IEEE reciprocal of every E4M3 scale; 0 for scale 0 (and NaN codes)
         const float v = e4m3_value(threadIdx.x);
-        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] = (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
+        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] =
+            (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
     }
-    if (warp == kWarpMma) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -245,100 +225,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const float *rcp_lut = reinterpret_cast<const float *>(base + C::oLut);
 
-    if (warp >= kWarpCorr) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCorr));
-        // ---------------------------------------- O correction + epilogue
-        // Thread = row r of both tiles (TMEM lane r).  For every KV block
-        // j >= 1 of tile i: O_i *= alpha_i(j) after P V of block j-1 has
-        // completed and before P V of block j is issued.
-        const int wq = warp & 3;
-        const int r = wq * 32 + lane;
-        const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        const float *alpha_buf = reinterpret_cast<const float *>(base + C::oAlpha);
-        const float *l_buf = reinterpret_cast<const float *>(base + C::oL);
-        bool ok = true;
-        for (int j = 1; ok && j < nmax; ++j) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (j >= (i ? n1 : n0)) continue;
-                if (!warp_wait(bars + kBarAlpha + 2 * i + (j & 1), ((j - 1) >> 1) & 1, abort_flag) ||
-                    !warp_wait(bars + kBarPvDone + 2 * i + ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const float alpha = alpha_buf[(2 * i + (j & 1)) * 128 + r];
-                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                    const uint32_t tO = i ? C::tO1 : C::tO0;
-                    const uint64_t aa = pack2(alpha, alpha);
-#pragma unroll
-                    for (int q = 0; q < D / 32; ++q) {
-                        uint32_t o[32];
-                        tmem_ld32(trow + tO + 32 * q, o);
-                        tmem_ld_wait();
-                        reg_fence32(o);
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const uint64_t v = mul2(pack2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa);
-                            o[e] = __float_as_uint(lo2(v));
-                            o[e + 1] = __float_as_uint(hi2(v));
-                        }
-                        tmem_st32(trow + tO + 32 * q, o);
-                    }
-                    tmem_st_wait();
-                }
-                tc_fence_before();
-                mbar_arrive(bars + kBarCorr + i);
-            }
-        }
-        // epilogue: out = bf16(O / l) for rows < N
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int n_i = i ? n1 : n0;
-            if (!ok || n_i == 0) continue;
-            if (!warp_wait(bars + kBarL + i, 0, abort_flag) ||
-                !warp_wait(bars + kBarPvDone + 2 * i + ((n_i - 1) & 1), ((n_i - 1) >> 1) & 1, abort_flag)) {
-                ok = false;
-                continue;
-            }
-            tc_fence_after();
-            const float inv = __frcp_rn(l_buf[i * 128 + r]);
-            const int grow = (i ? tile1 : tile0) * kBlk + r;
-            const uint32_t tO = i ? C::tO1 : C::tO0;
-            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.N + grow) * D;
-#pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t o[32];
-                tmem_ld32(trow + tO + 32 * q, o);
-                tmem_ld_wait();
-                reg_fence32(o);
-                if (grow < p.N) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
-                                                                        __uint_as_float(o[2 * e + 1]) * inv);
-                        w[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * q);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-                }
-            }
-        }
-    } else if (warp >= kWarpProducer) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLoad));
-      if (warp == kWarpProducer) {
+    if (warp >= 8) {
+      if (warp == 8) {
         // ------------------------------------------------------ producer
-        // The whole warp runs the loop (uniform values); one elected lane
-        // issues the copies.
-        const bool leader = elect_one();
-        uint64_t *bq = bars + kBarQ;
-        if (leader) {
+        if (lane == 0) {
             prefetch_tensormap(&tm_q);
             prefetch_tensormap(&tm_k);
             prefetch_tensormap(&tm_v);
+            uint64_t *bq = bars + kBarQ;
             mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * (C::kQBytes + C::kSfBytes));
             tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Np + tile0 * kBlk, bq);
             bulk_load(base + C::oQsf0, p.q_sf + static_cast<size_t>(bh * nqt + tile0) * C::kSfBytes, C::kSfBytes, bq);
@@ -347,76 +243,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bulk_load(base + C::oQsf1, p.q_sf + static_cast<size_t>(bh * nqt + tile1) * C::kSfBytes, C::kSfBytes,
                           bq);
             }
-        }
-        __syncwarp();
-        int issued = 0;
-        for (int j = 0; j < nmax; ++j) {
-            const int s = j % kStages;
-            const int u = j / kStages;
-            if (u > 0 && !warp_wait(bars + kBarKvEmpty + s, (u - 1) & 1, abort_flag)) break;
-            uint8_t *st = base + C::oStage + s * C::kStageBytes;
-            uint64_t *bf = bars + kBarKvFull + s;
-            if (leader) {
+            int issued = 0;
+            for (int j = 0; j < nmax; ++j) {
+                const int s = j % kStages;
+                const int u = j / kStages;
+                if (u > 0 && !mbar_wait(bars + kBarKvEmpty + s, (u - 1) & 1, abort_flag)) break;
+                uint8_t *st = base + C::oStage + s * C::kStageBytes;
+                uint64_t *bf = bars + kBarKvFull + s;
                 mbar_arrive_expect_tx(bf, C::kQBytes + C::kSfBytes + C::kVBytes + C::kVsfBytes);
                 tma_load_2d(st + C::sK, &tm_k, 0, bh * p.Np + j * kBlk, bf);
                 bulk_load(st + C::sKsf, p.k_sf + static_cast<size_t>(bh * nqt + j) * C::kSfBytes, C::kSfBytes, bf);
                 tma_load_2d(st + C::sV, &tm_v, j * 64, bh * D, bf);
                 bulk_load(st + C::sVsf, p.vt_sf + (static_cast<size_t>(bh) * (p.Np / 64) + 2 * j) * 512, C::kVsfBytes,
                           bf);
+                issued = j + 1;
             }
-            __syncwarp();
-            issued = j + 1;
+            // Let every copy this thread started land before the CTA exits.
+            drain_wait(bq, 0);
+            for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
+                drain_wait(bars + kBarKvFull + j % kStages, (j / kStages) & 1);
         }
-        // Let every copy this warp started land before the CTA exits.
-        drain_wait(bq, 0);
-        for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
-            drain_wait(bars + kBarKvFull + j % kStages, (j / kStages) & 1);
-      } else if (warp == kWarpMma) {
+    } else if (warp == 9) {
         // ----------------------------------------------------------- MMA
-        // The whole warp runs the loop, so addresses and descriptors stay in
-        // uniform registers; one elected lane issues each tcgen05 op.
-        const bool leader = elect_one();
-        constexpr uint32_t idesc_qk = idesc_mxf4nvf4(128, 128);
-        constexpr uint32_t idesc_pv = idesc_mxf4nvf4(128, D);
-        int nqk = 0;
-        auto stage_s = [&](int j) -> uint32_t {
-            return base_s + C::oStage + static_cast<uint32_t>(j % kStages) * C::kStageBytes;
-        };
-        auto copy_ksf = [&](int j) {
-            if (leader) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_mxf4nvf4(128, 128);
+            constexpr uint32_t idesc_pv = idesc_mxf4nvf4(128, D);
+            int nqk = 0;
+            auto stage_s = [&](int j) -> uint32_t {
+                return base_s + C::oStage + static_cast<uint32_t>(j % kStages) * C::kStageBytes;
+            };
+            auto copy_ksf = [&](int j) {
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a)
                     tc_cp_32x128b_warpx4(tmem + C::tSfk + 4 * a, sdesc_sf_atom(stage_s(j) + C::sKsf + 512 * a));
-            }
-            __syncwarp();
-        };
-        auto issue_qk = [&](int i, int j) -> bool {
-            if (nqk > 0 && !warp_wait(bars + kBarSEmpty, (nqk - 1) & 1, abort_flag)) return false;
-            tc_fence_after();
-            const uint32_t qa = base_s + (i ? C::oQ1 : C::oQ0);
-            const uint32_t kb = stage_s(j) + C::sK;
-            if (leader) {
+            };
+            auto issue_qk = [&](int i, int j) -> bool {
+                if (nqk > 0 && !mbar_wait(bars + kBarSEmpty, (nqk - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t qa = base_s + (i ? C::oQ1 : C::oQ0);
+                const uint32_t kb = stage_s(j) + C::sK;
 #pragma unroll
                 for (int kc = 0; kc < D / 64; ++kc)
                     tc_mma_mxf4nvf4(tmem + C::tS, sdesc_kmajor_sw(qa + 32 * kc, C::kQKSbo, C::kQKLayout),
                                     sdesc_kmajor_sw(kb + 32 * kc, C::kQKSbo, C::kQKLayout), idesc_qk,
                                     tmem + (i ? C::tSfq1 : C::tSfq0) + 4 * kc, tmem + C::tSfk + 4 * kc, kc > 0);
                 tc_commit(bars + kBarSFull + i);
-            }
-            __syncwarp();
-            ++nqk;
-            return true;
-        };
-        auto issue_pv = [&](int i, int j, bool load_vsf) -> bool {
-            if (!warp_wait(bars + kBarPFull + 2 * i + (j & 1), (j >> 1) & 1, abort_flag)) return false;
-            if (j > 0 && !warp_wait(bars + kBarCorr + i, (j - 1) & 1, abort_flag)) return false;
-            tc_fence_after();
-            const uint32_t buf = static_cast<uint32_t>(2 * i + (j & 1));
-            const uint32_t pa = base_s + C::oP + buf * C::kPBytes;
-            const uint32_t psf = base_s + C::oPsf + buf * C::kPsfBytes;
-            const uint32_t vb = stage_s(j) + C::sV;
-            const uint32_t vsf = stage_s(j) + C::sVsf;
-            if (leader) {
+                ++nqk;
+                return true;
+            };
+            auto issue_pv = [&](int i, int j, bool load_vsf) -> bool {
+                if (!mbar_wait(bars + kBarPFull + i, j & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t pa = base_s + (i ? C::oP1 : C::oP0);
+                const uint32_t psf = base_s + (i ? C::oPsf1 : C::oPsf0);
+                const uint32_t vb = stage_s(j) + C::sV;
+                const uint32_t vsf = stage_s(j) + C::sVsf;
                 tc_cp_32x128b_warpx4(tmem + C::tSfp, sdesc_sf_atom(psf));
                 tc_cp_32x128b_warpx4(tmem + C::tSfp + 4, sdesc_sf_atom(psf + 512));
                 if (load_vsf) {
@@ -428,53 +309,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_mxf4nvf4(tmem + (i ? C::tO1 : C::tO0), sdesc_kmajor_sw(pa + 32 * kc, 512, 4u),
                                     sdesc_kmajor_sw(vb + 32 * kc, 512, 4u), idesc_pv, tmem + C::tSfp + 4 * kc,
                                     tmem + C::tSfv + 4 * kc, (j > 0 || kc > 0) ? 1u : 0u);
-                tc_commit(bars + kBarPvDone + buf);
-            }
-            __syncwarp();
-            return true;
-        };
+                tc_commit(bars + kBarPvDone + i);
+                return true;
+            };
 
-        bool ok = warp_wait(bars + kBarQ, 0, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            if (leader) {
+            bool ok = mbar_wait(bars + kBarQ, 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a) {
                     tc_cp_32x128b_warpx4(tmem + C::tSfq0 + 4 * a, sdesc_sf_atom(base_s + C::oQsf0 + 512 * a));
                     if (valid1)
                         tc_cp_32x128b_warpx4(tmem + C::tSfq1 + 4 * a, sdesc_sf_atom(base_s + C::oQsf1 + 512 * a));
                 }
+                ok = mbar_wait(bars + kBarKvFull + 0, 0, abort_flag);
             }
-            __syncwarp();
-            ok = warp_wait(bars + kBarKvFull + 0, 0, abort_flag);
-        }
-        if (ok) {
-            tc_fence_after();
-            copy_ksf(0);
-            if (n0 > 0) ok = issue_qk(0, 0);
-            if (ok && n1 > 0) ok = issue_qk(1, 0);
-        }
-        for (int j = 0; ok && j < nmax; ++j) {
-            if (j + 1 < nmax) {
-                ok = warp_wait(bars + kBarKvFull + (j + 1) % kStages, ((j + 1) / kStages) & 1, abort_flag);
-                if (!ok) break;
+            if (ok) {
                 tc_fence_after();
-                copy_ksf(j + 1);
+                copy_ksf(0);
+                if (n0 > 0) ok = issue_qk(0, 0);
+                if (ok && n1 > 0) ok = issue_qk(1, 0);
             }
-            if (j + 1 < n0 && !(ok = issue_qk(0, j + 1))) break;
-            if (j < n0 && !(ok = issue_pv(0, j, true))) break;
-            if (j + 1 < n1 && !(ok = issue_qk(1, j + 1))) break;
-            if (j < n1 && !(ok = issue_pv(1, j, !(j < n0)))) break;
-            if (leader) tc_commit(bars + kBarKvEmpty + j % kStages);
-            __syncwarp();
+            for (int j = 0; ok && j < nmax; ++j) {
+                if (j + 1 < nmax) {
+                    ok = mbar_wait(bars + kBarKvFull + (j + 1) % kStages, ((j + 1) / kStages) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    copy_ksf(j + 1);
+                }
+                if (j + 1 < n0 && !(ok = issue_qk(0, j + 1))) break;
+                if (j < n0 && !(ok = issue_pv(0, j, true))) break;
+                if (j + 1 < n1 && !(ok = issue_qk(1, j + 1))) break;
+                if (j < n1 && !(ok = issue_pv(1, j, !(j < n0)))) break;
+                tc_commit(bars + kBarKvEmpty + j % kStages);
+            }
+            // Every tcgen05 op issued above completes before TMEM is freed.
+            tc_commit(bars + kBarDrain);
+            drain_wait(bars + kBarDrain, 0);
         }
-        // Every tcgen05 op issued above completes before TMEM is freed.
-        if (leader) tc_commit(bars + kBarDrain);
         __syncwarp();
-        drain_wait(bars + kBarDrain, 0);
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ------------------------------------------------------- softmax
         const int i = warp >> 2;       // Q tile of this warpgroup
         const int wq = warp & 3;       // TMEM sub-partition = rows 32*wq ..
@@ -484,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_i = i ? n1 : n0;
         const float c2 = p.scale_log2;
         const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        const float *rcp_lut = reinterpret_cast<const float *>(base + C::oLut);
-        float *alpha_buf = reinterpret_cast<float *>(base + C::oAlpha);
+        const uint32_t tO = i ? C::tO1 : C::tO0;
+        uint8_t *P = base + (i ? C::oP1 : C::oP0);
+        uint8_t *Psf = base + (i ? C::oPsf1 : C::oPsf0);
         float m = -INFINITY;
         float l = 0.0f;
         bool ok = true;
@@ -534,11 +410,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float m_new = fmaxf(m, __fmul_rn(rmax, c2));
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
-            if (j > 0) {
-                // hand alpha to the correction warpgroup right away
-                alpha_buf[(2 * i + (j & 1)) * 128 + r] = alpha;
-                mbar_arrive(bars + kBarAlpha + 2 * i + (j & 1));
-            }
             // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
             // two blocks per conversion; r_b = 1/s_b from the exact table
             uint32_t scw[2];
@@ -563,9 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t *x = &s[b >> 1][(b & 1) * 16];
                 uint64_t vp[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), cc, nn);
-                    vp[e] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
+                for (int i = 0; i < 8; ++i) {
+                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), cc, nn);
+                    vp[i] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
                 }
                 const uint64_t s01 = add2(add2(vp[0], vp[1]), add2(vp[2], vp[3]));
                 const uint64_t s23 = add2(add2(vp[4], vp[5]), add2(vp[6], vp[7]));
@@ -573,46 +444,89 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t rr = pack2(rb[b], rb[b]);
                 uint64_t vy[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) vy[e] = mul2(vp[e], rr);
+                for (int i = 0; i < 8; ++i) vy[i] = mul2(vp[i], rr);
                 pc[2 * b] = cvt_e2m1x8(lo2(vy[0]), hi2(vy[0]), lo2(vy[1]), hi2(vy[1]), lo2(vy[2]), hi2(vy[2]),
                                        lo2(vy[3]), hi2(vy[3]));
                 pc[2 * b + 1] = cvt_e2m1x8(lo2(vy[4]), hi2(vy[4]), lo2(vy[5]), hi2(vy[5]), lo2(vy[6]), hi2(vy[6]),
                                            lo2(vy[7]), hi2(vy[7]));
             }
-            l = alpha * l + (lo2(acc) + hi2(acc));
+            const float sum = lo2(acc) + hi2(acc);
+            const uint32_t scw0 = scw[0], scw1 = scw[1];
+            l = alpha * l + sum;
 
-            // P buffer (j & 1) is free once P V of block j-2 has completed.
-            const int buf = 2 * i + (j & 1);
-            if (j >= 2) {
-                if (!warp_wait(bars + kBarPvDone + buf, ((j - 2) >> 1) & 1, abort_flag)) {
+            // P buffer and O are free once the previous P V has completed.
+            if (j > 0) {
+                if (!warp_wait(bars + kBarPvDone + i, (j - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
+                tc_fence_after();
             }
             {
-                uint8_t *prow = base + C::oP + buf * C::kPBytes + (r >> 3) * 512 + (r & 7) * 64;
-                uint8_t *psf = base + C::oPsf + buf * C::kPsfBytes;
+                uint8_t *prow = P + (r >> 3) * 512 + (r & 7) * 64;
                 const int sw = (r & 7) >> 1;
 #pragma unroll
                 for (int c16 = 0; c16 < 4; ++c16)
                     *reinterpret_cast<uint4 *>(prow + ((c16 ^ sw) << 4)) =
                         make_uint4(pc[4 * c16], pc[4 * c16 + 1], pc[4 * c16 + 2], pc[4 * c16 + 3]);
-                *reinterpret_cast<uint32_t *>(psf + 16 * (r & 31) + 4 * (r >> 5)) = scw[0];
-                *reinterpret_cast<uint32_t *>(psf + 512 + 16 * (r & 31) + 4 * (r >> 5)) = scw[1];
+                *reinterpret_cast<uint32_t *>(Psf + 16 * (r & 31) + 4 * (r >> 5)) = scw0;
+                *reinterpret_cast<uint32_t *>(Psf + 512 + 16 * (r & 31) + 4 * (r >> 5)) = scw1;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                // O = alpha * O for this warp's 32 rows
+                uint32_t o[D / 32][32];
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
+                tmem_ld_wait();
+#pragma unroll
+                const uint64_t aa = pack2(alpha, alpha);
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    reg_fence32(o[q]);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const uint64_t v = mul2(pack2(__uint_as_float(o[q][e]), __uint_as_float(o[q][e + 1])), aa);
+                        o[q][e] = __float_as_uint(lo2(v));
+                        o[q][e + 1] = __float_as_uint(hi2(v));
+                    }
+                    tmem_st32(trow + tO + 32 * q, o[q]);
+                }
+                tmem_st_wait();
             }
             fence_proxy_async_smem();
-            mbar_arrive(bars + kBarPFull + buf);
+            tc_fence_before();
+            mbar_arrive(bars + kBarPFull + i);
             m = m_new;
         }
-        if (ok && n_i > 0) {
-            reinterpret_cast<float *>(base + C::oL)[i * 128 + r] = l;
-            mbar_arrive(bars + kBarL + i);
+        if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
+            tc_fence_after();
+            const float inv = __frcp_rn(l);
+            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.N + grow) * D;
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t o[32];
+                tmem_ld32(trow + tO + 32 * q, o);
+                tmem_ld_wait();
+                reg_fence32(o);
+                if (grow < p.N) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                                        __uint_as_float(o[2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * q);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kWarpMma) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

@@ -13,7 +13,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/sa3.h"
+#include "sa3.h"
 #include "sa3_internal.h"
 #include "sm100.cuh"
 

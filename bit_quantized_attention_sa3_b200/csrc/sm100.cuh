@@ -73,14 +73,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware park the thread for up to `hint_ns`
+// while the phase is incomplete (no busy polling).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+#ifndef SA3_WAIT_HINT_NS
+#define SA3_WAIT_HINT_NS 1000000
+#endif
+
 // Wait for the phase of `bar` with the given parity to complete.  Bounded:
 // gives up after kWaitLimitNs or as soon as *abort is set by another warp;
 // on giving up it records the timeout and sets *abort.  Returns success.
+// The thread sleeps inside try_wait (suspend hint) instead of spinning, so
+// waiting warps take no issue slots from the working ones.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_hint(bar, parity, SA3_WAIT_HINT_NS)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort = 1;
