@@ -80,8 +80,14 @@ def padded_len(N: int) -> int:
     return (N + BLK - 1) // BLK * BLK
 
 
+def kmean_chunk(N: int) -> int:
+    return 512 * (((N + 511) // 512 + 15) // 16)
+
+
 def quant_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
-    return B * H * ((N + 511) // 512) * d * 8
+    """sa3_quant_workspace_bytes of include/sa3.h."""
+    c = kmean_chunk(N)
+    return B * H * ((N + c - 1) // c) * d * 8
 
 
 @dataclasses.dataclass

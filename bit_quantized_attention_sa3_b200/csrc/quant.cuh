@@ -9,10 +9,12 @@
 // E2M1_RN_sat(x_i * r), all zero if s == 0 -- see include/sa3.h.
 //
 // HBM-bound streaming work, three launches on the caller's stream:
-//   A  Q tiles, V tiles (transposed through shared memory), and per-512-
-//      token fp64 partial sums of K, ordered so that K is read last;
-//   B  one CTA per (b, h): partial sums -> mean (fixed order, fp64);
-//   C  K tiles, smoothed with the mean (K re-read, from L2 when it fits).
+//   A  Q tiles, V tiles (transposed through shared memory), and fp64
+//      partial sums of K over at most 16 token chunks per (b, h), ordered so
+//      that K is read last;
+//   B  K tiles: each CTA first adds its (b, h)'s partial sums in chunk order
+//      (fp64) into the mean, then smooths and quantizes its tile (K re-read,
+//      from L2 when it fits).
 // Q/K tiles: two threads per 16-element block, one 128-bit load each,
 // block amax combined with one warp shuffle.  V tiles: a 128-token tile
 // is staged in shared memory with a 16-byte XOR swizzle so that the
@@ -169,7 +171,7 @@ __device__ __forceinline__ void v_tile(const __nv_bfloat16 *__restrict__ src, in
 
 // fp64 partial sums of K over one 512-token chunk.
 template <int D>
-__device__ __forceinline__ void k_partial(const __nv_bfloat16 *__restrict__ src, int N, int chunk,
+__device__ __forceinline__ void k_partial(const __nv_bfloat16 *__restrict__ src, int N, int chunk, int chunk_len,
                                           double *__restrict__ part, double *red) {
     constexpr int kVec = D / 8;
     constexpr int kRows = kThreads / kVec;  // rows covered per step
@@ -179,8 +181,8 @@ __device__ __forceinline__ void k_partial(const __nv_bfloat16 *__restrict__ src,
     double acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-    const int t0 = chunk * kQuantChunk;
-    const int t1 = min(N, t0 + kQuantChunk);
+    const int t0 = chunk * chunk_len;
+    const int t1 = min(N, t0 + chunk_len);
     constexpr int kBatch = 8;
     for (int tb = t0 + r0; tb < t1; tb += kRows * kBatch) {
         uint4 raw[kBatch];
@@ -208,7 +210,7 @@ __device__ __forceinline__ void k_partial(const __nv_bfloat16 *__restrict__ src,
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) quant_qv_ksum_kernel(QuantParams p) {
+__global__ void __launch_bounds__(kThreads, 4) quant_qv_ksum_kernel(QuantParams p) {
     __shared__ __align__(16) uint8_t smem[kTile * D * 2];
     const int bh = blockIdx.y;
     const int x = blockIdx.x;
@@ -222,26 +224,25 @@ __global__ void __launch_bounds__(kThreads) quant_qv_ksum_kernel(QuantParams p) 
                   p.vt_sf + static_cast<size_t>(bh) * p.Np * 8, reinterpret_cast<uint32_t *>(smem));
     } else {  // K partial sums
         if (x >= p.nchunk) return;
-        k_partial<D>(p.k + in_off, p.N, x, p.part + static_cast<size_t>(bh) * p.nchunk * D,
+        k_partial<D>(p.k + in_off, p.N, x, p.chunk, p.part + static_cast<size_t>(bh) * p.nchunk * D,
                      reinterpret_cast<double *>(smem));
     }
-}
-
-template <int D>
-__global__ void __launch_bounds__(D) kmean_finalize_kernel(QuantParams p) {
-    const int bh = blockIdx.x;
-    const int c = threadIdx.x;
-    double s = 0.0;
-    const double *part = p.part + static_cast<size_t>(bh) * p.nchunk * D;
-    for (int ch = 0; ch < p.nchunk; ++ch) s += part[static_cast<size_t>(ch) * D + c];
-    p.k_mean[static_cast<size_t>(bh) * D + c] = __double2float_rn(s / static_cast<double>(p.N));
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) quant_k_kernel(QuantParams p) {
     __shared__ float mean[D];
     const int bh = blockIdx.y;
-    for (int c = threadIdx.x; c < D; c += kThreads) mean[c] = p.k_mean[static_cast<size_t>(bh) * D + c];
+    // mean of K over its N tokens: partial sums added in chunk order (fp64),
+    // one division, one rounding to fp32; tile 0 also stores it
+    for (int c = threadIdx.x; c < D; c += kThreads) {
+        const double *part = p.part + static_cast<size_t>(bh) * p.nchunk * D + c;
+        double s = 0.0;
+        for (int ch = 0; ch < p.nchunk; ++ch) s += part[static_cast<size_t>(ch) * D];
+        const float mu = __double2float_rn(s / static_cast<double>(p.N));
+        mean[c] = mu;
+        if (blockIdx.x == 0) p.k_mean[static_cast<size_t>(bh) * D + c] = mu;
+    }
     __syncthreads();
     qk_tile<D, true>(p.k + static_cast<size_t>(bh) * p.N * D, p.N, blockIdx.x, mean,
                      p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
@@ -252,7 +253,6 @@ template <int D>
 cudaError_t launch_quant_d(const QuantParams &p, cudaStream_t stream) {
     const int ntile = p.Np / kTile;
     quant_qv_ksum_kernel<D><<<dim3(ntile, p.BH, 3), kThreads, 0, stream>>>(p);
-    kmean_finalize_kernel<D><<<p.BH, D, 0, stream>>>(p);
     quant_k_kernel<D><<<dim3(ntile, p.BH, 1), kThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }

@@ -75,6 +75,21 @@ int check_qkv(const sa3_qkv_fp4 *t) {
     return SA3_OK;
 }
 
+// Self-test of the bounded waits: one warp waits on an mbarrier that nothing
+// ever arrives on, through the same routine the attention kernel uses, so
+// the wait must give up after `limit_ns` and record the timeout.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        sa3::mbar_init(&bar, 1);
+        abort_flag = 0;
+        sa3::fence_mbar_init();
+    }
+    __syncwarp();
+    sa3::mbar_wait_limit(&bar, 0, &abort_flag, limit_ns);
+}
+
 // Scratch for sa3_quantize_qkv_noalloc: one fixed array per device that
 // loads the library (fp64 K-mean partial sums).
 static __device__ __align__(256) double g_noalloc_scratch[SA3_NOALLOC_SCRATCH_BYTES / sizeof(double)];
@@ -125,7 +140,8 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, 
     p.BH = B * H;
     p.N = N;
     p.Np = static_cast<int>(sa3_padded_len(N));
-    p.nchunk = (N + sa3::kQuantChunk - 1) / sa3::kQuantChunk;
+    p.chunk = static_cast<int>(sa3_kmean_chunk(N));
+    p.nchunk = static_cast<int>(sa3_kmean_nchunk(N));
     return sa3::launch_quant(p, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK : SA3_ERR_CUDA;
 }
 
@@ -173,6 +189,13 @@ int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, 
     return sa3::launch_attn(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA3_OK
                : SA3_ERR_CUDA;
+}
+
+int sa3_selftest_wait_timeout(unsigned int limit_us, struct CUstream_st *stream) {
+    if (limit_us == 0 || limit_us > 10u * 1000u * 1000u) return SA3_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(limit_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? SA3_OK : SA3_ERR_CUDA;
 }
 
 int sa3_device_status(struct CUstream_st *stream) {

@@ -8,7 +8,6 @@
 
 namespace sa3 {
 
-constexpr int kQuantChunk = 512;  // tokens per fp64 partial sum of K
 
 struct QuantParams {
     const __nv_bfloat16 *q;
@@ -25,7 +24,8 @@ struct QuantParams {
     int BH;
     int N;
     int Np;
-    int nchunk;
+    int nchunk;  // fp64 partial sums of K per (b, h)
+    int chunk;   // tokens per partial sum
 };
 
 struct AttnParams {

@@ -92,22 +92,26 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parit
 #endif
 
 // Wait for the phase of `bar` with the given parity to complete.  Bounded:
-// gives up after kWaitLimitNs or as soon as *abort is set by another warp;
-// on giving up it records the timeout and sets *abort.  Returns success.
-// The thread sleeps inside try_wait (suspend hint) instead of spinning, so
+// gives up after `limit_ns` or as soon as *abort is set by another warp; on
+// giving up it records the timeout and sets *abort.  Returns success.  The
+// thread sleeps inside try_wait (suspend hint) instead of spinning, so
 // waiting warps take no issue slots from the working ones.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait_hint(bar, parity, SA3_WAIT_HINT_NS)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort = 1;
             atomicOr(&g_sa3_status, 1u);
             return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait_limit(bar, parity, abort, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------ TMA / bulk

@@ -97,9 +97,13 @@ static inline int64_t sa3_vt_fp4_bytes(int64_t B, int64_t H, int64_t N, int64_t 
 static inline int64_t sa3_vt_sf_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
 { (void)d; return B * H * sa3_padded_len(N) * 8; }
 static inline int64_t sa3_kmean_bytes(int64_t B, int64_t H, int64_t d) { return B * H * d * 4; }
-/* Scratch for the K-mean reduction: fp64 partial sums per 512 tokens. */
+/* Scratch for the K-mean reduction: fp64 partial sums over chunks of
+ * sa3_kmean_chunk(N) tokens (a multiple of 512 chosen so that there are at
+ * most 16 chunks). */
+static inline int64_t sa3_kmean_chunk(int64_t N) { return 512 * (((N + 511) / 512 + 15) / 16); }
+static inline int64_t sa3_kmean_nchunk(int64_t N) { return (N + sa3_kmean_chunk(N) - 1) / sa3_kmean_chunk(N); }
 static inline int64_t sa3_quant_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
-{ return B * H * ((N + 511) / 512) * d * 8; }
+{ return B * H * sa3_kmean_nchunk(N) * d * 8; }
 
 /*
  * sa3_quantize_qkv -- K smoothing plus FP4 microscaling of Q, K and V.
@@ -164,7 +168,8 @@ int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d,
  * library holds in device memory on every GPU that loads it, until the
  * process exits.  The array holds SA3_NOALLOC_SCRATCH_BYTES bytes, so the
  * call accepts shapes with sa3_quant_workspace_bytes(B, H, N, d) <=
- * SA3_NOALLOC_SCRATCH_BYTES and returns SA3_ERR_UNSUPPORTED otherwise.
+ * SA3_NOALLOC_SCRATCH_BYTES (at most 16 chunks, so B*H*d <= 32768) and
+ * returns SA3_ERR_UNSUPPORTED otherwise.
  * It calls no allocation routine.
  *
  * The first call on a device looks up that device's copy of the array
@@ -188,6 +193,17 @@ int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v,
  * else SA3_OK.
  */
 int sa3_device_status(struct CUstream_st *stream);
+
+/*
+ * sa3_selftest_wait_timeout -- exercises the failure path of the bounded
+ * device waits: enqueues one warp that waits, through the same routine the
+ * kernels above use, on a barrier nothing arrives on, for `limit_us`
+ * microseconds (1 .. 10^7).  The wait gives up, records SA3_ERR_TIMEOUT in
+ * the status word and the kernel returns; the CUDA context stays usable.
+ * A following sa3_device_status() returns SA3_ERR_TIMEOUT (and clears it).
+ * No counterpart in the method; for tests of failure detection.
+ */
+int sa3_selftest_wait_timeout(unsigned int limit_us, struct CUstream_st *stream);
 
 /* Library version string, e.g. "libsa3 0.1.0 (sm_100a)". Host memory,
  * static, never freed. */

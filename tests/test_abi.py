@@ -27,7 +27,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert _declared() == ["sa3_attn_fwd", "sa3_device_status", "sa3_quantize_qkv",
-                           "sa3_quantize_qkv_noalloc", "sa3_version"]
+                           "sa3_quantize_qkv_noalloc", "sa3_selftest_wait_timeout", "sa3_version"]
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -55,3 +55,6 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.sa3_attn_fwd(None, 1, 1, 8, 100, 0, 0.0, None, None) == 2
     # B*H beyond the grid limit
     assert lib.sa3_attn_fwd(None, 1000, 1000, 8, 64, 0, 0.0, None, None) == 2
+    lib.sa3_selftest_wait_timeout.restype = I
+    lib.sa3_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
+    assert lib.sa3_selftest_wait_timeout(0, None) == 1
