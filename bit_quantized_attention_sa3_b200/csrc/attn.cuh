@@ -182,14 +182,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;
+    // Work unit -> (b*H+h, Q tiles).  Units [0, pair_units) are pairs of
+    // Q tiles, ordered by rank (heaviest pairs first when causal) and then
+    // head; the pairs after them are split into single-tile units that fill
+    // what would otherwise be a short last wave.
     const int nqt = p.Np / kBlk;
-    // causal: heaviest Q-tile pairs first
-    const int pair = p.causal ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
-                              : static_cast<int>(blockIdx.x);
-    const int tile0 = 2 * pair;
-    const int tile1 = 2 * pair + 1;
-    const bool valid1 = tile1 < nqt;
+    const int u = static_cast<int>(blockIdx.x);
+    const bool single = u >= p.pair_units;
+    const int pu = single ? p.pair_units + (u - p.pair_units) / 2 : u;
+    const int bh = pu % p.BH;
+    const int rank = pu / p.BH;
+    const int pair = p.causal ? p.npairs - 1 - rank : rank;
+    const int tile0 = 2 * pair + (single ? ((u - p.pair_units) & 1) : 0);
+    const int tile1 = tile0 + 1;
+    if (tile0 >= nqt) return;  // second half of a split pair whose head has an odd tile count
+    const bool valid1 = !single && tile1 < nqt;
     const int n0 = p.causal ? tile0 + 1 : nqt;
     const int n1 = valid1 ? (p.causal ? tile1 + 1 : nqt) : 0;
     const int nmax = n0 > n1 ? n0 : n1;
@@ -539,9 +546,19 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // Split the pairs of a last wave that would fill at most half of the SMs
+    // into single-tile units (one CTA per SM).
+    AttnParams q = p;
     const int nqt = p.Np / kBlk;
-    const dim3 grid((nqt + 1) / 2, p.BH);
-    attn_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    q.npairs = (nqt + 1) / 2;
+    const int total = q.npairs * p.BH;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int rem = total % nsm;
+    const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
+    q.pair_units = total - split;
+    const dim3 grid(q.pair_units + 2 * split);
+    attn_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
     return cudaGetLastError();
 }
 

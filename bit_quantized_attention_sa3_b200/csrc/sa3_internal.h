@@ -38,6 +38,8 @@ struct AttnParams {
     int Np;
     int causal;
     float scale_log2;  // fp32(sm_scale * log2 e)
+    int npairs;        // Q-tile pairs per head (set by the launcher)
+    int pair_units;    // work units that are pairs; the rest are single tiles
 };
 
 }  // namespace sa3

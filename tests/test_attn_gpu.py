@@ -133,3 +133,15 @@ def test_attn_rejects_bad_arguments():
     with pytest.raises(sa3.Sa3Error) as e:
         sa3.attn_fwd(qz, out=mis)
     assert e.value.code == sa3.SA3_ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["noncausal", "causal"])
+def test_attn_tail_wave_single_tile_units(causal):
+    """151 heads x 3 Q tiles = 302 tile pairs: the pairs of the short last
+    wave run as single-tile work units; every row must still match."""
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("split point assumes 148 SMs")
+    err, cos_gpu, cos_oracle = _run("tiny_b1h2n256d64", {"H": 151, "N": 300}, causal)
+    assert err <= TOL, f"rel-L2 vs oracle {err:.3e}"
+    assert cos_gpu >= cos_oracle - 1e-3
