@@ -1,4 +1,4 @@
-// quant.cu -- K smoothing and FP4 microscaling of Q, K and V.
+// quant.cuh -- K smoothing and FP4 microscaling of Q, K and V.
 //
 // Method: "SageAttention: Accurate 8-Bit Attention for Plug-and-play
 // Inference Acceleration" (summary, section "Approach") smooths K by
@@ -8,259 +8,558 @@
 // block (x_0..x_15):  s = E4M3_RN_sat(amax/6), r = 1/s, code_i =
 // E2M1_RN_sat(x_i * r), all zero if s == 0 -- see include/sa3.h.
 //
-// HBM-bound streaming work, three launches on the caller's stream:
-//   A  Q tiles, V tiles (transposed through shared memory), and fp64
-//      partial sums of K over at most 16 token chunks per (b, h), ordered so
-//      that K is read last;
-//   B  K tiles: each CTA first adds its (b, h)'s partial sums in chunk order
-//      (fp64) into the mean, then smooths and quantizes its tile (K re-read,
-//      from L2 when it fits).
-// Q/K tiles: two threads per 16-element block, one 128-bit load each,
-// block amax combined with one warp shuffle.  V tiles: a 128-token tile
-// is staged in shared memory with a 16-byte XOR swizzle so that the
-// column reads of the transpose are conflict-free.
+// HBM-bound streaming work in two launches on the caller's stream, both
+// made of persistent CTAs (two per SM) that stream 128-token bf16 tiles
+// through a ring of shared-memory buffers filled by 3-D TMA loads (64
+// channels x 128 tokens per box, 128-byte swizzle, rows past N zero-filled
+// by the copy engine):
+//   A  each CTA takes a balanced static share of the Q and V tiles and then
+//      of the K chunks (fp64 column sums of K over at most 16 token chunks
+//      per (b, h)); K comes last so that it is still in L2 for B;
+//   B  K tiles, launched as a programmatic dependent of A: each CTA starts
+//      its first K loads, waits for A, forms the mean of each (b, h) it
+//      meets from the chunk sums (in chunk order, fp64), then smooths and
+//      quantizes its contiguous range of tiles.
+// Thread layouts (256 threads per CTA), all conflict-free on the swizzled
+// tiles: Q/K tiles -- a thread owns D/32 consecutive 16-element blocks of
+// one token row; V tiles (quantized transposed, 16 tokens per block) -- a
+// thread owns a pair of channels over D/64 consecutive 16-token blocks,
+// warps reading 32 consecutive channel pairs of one token row at a time;
+// K sums -- a thread owns 8 channels of every 16th (D=128) or 32nd (D=64)
+// row and the warps' fp64 sums are added in a fixed order.
 #pragma once
 
 #include "sa3_internal.h"
 #include "sm100.cuh"
 
 namespace sa3 {
+namespace quant {
 
-namespace {
+constexpr int kTile = 128;      // tokens per tile
+constexpr int kThreads = 256;   // threads per CTA
+constexpr int kWarps = kThreads / 32;
+constexpr int kStages = 3;      // tile buffers per CTA
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxChunks = 16;  // sa3_kmean_chunk keeps the chunk count at or below this
+constexpr int kBoxCh = 64;      // channels per TMA box (128 bytes of bf16)
 
-constexpr int kTile = 128;    // tokens per Q/K/V tile
-constexpr int kThreads = 256;  // threads per quantizer CTA
+template <int D>
+struct QCfg {
+    static constexpr int kBoxBytes = kTile * kBoxCh * 2;  // 16 KB
+    static constexpr int kTileBytes = kTile * D * 2;      // D/64 boxes
+    static constexpr int oStage = 0;
+    static constexpr int oRed = kStages * kTileBytes;     // fp64 K sums: one row of D per warp
+    static constexpr int oLut = oRed + kWarps * D * 8;    // 256 floats: 1 / E4M3 value
+    static constexpr int oMean = oLut + 256 * 4;          // -mean of K, D floats
+    static constexpr int oBar = oMean + D * 4;            // kStages full barriers + abort flag
+    static constexpr int kSmemBytes = oBar + kStages * 8 + 16 + 1024;  // + alignment slack
+};
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ void bf16x8(const uint4 &v, float (&x)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+// Byte offset of bf16 element (row, ch) inside a staged tile: box ch/64,
+// 128-byte rows, 16-byte chunk index XOR (row % 8) (128-byte swizzle).
+__device__ __forceinline__ int tile_off(int row, int ch) {
+    return (ch >> 6) * (kTile * kBoxCh * 2) + row * 128 + ((((ch & 63) >> 3) ^ (row & 7)) << 4) + (ch & 7) * 2;
 }
 
 // Byte offset of scale column c4 (0..3) of token-row r (0..127) inside a
 // 512-byte scale atom.
 __device__ __forceinline__ int atom_off(int r, int c4) { return 16 * (r & 31) + 4 * (r >> 5) + c4; }
 
-// Scale code and 1/scale of a block with the given amax (>= 0).
-__device__ __forceinline__ uint32_t block_scale(float amax, float &rcp) {
-    const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, 6.0f));
-    const float s = e4m3_value(sc);
-    rcp = (s == 0.0f) ? 0.0f : __frcp_rn(s);
-    return sc;
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Exact 1/s for every E4M3 scale code s (0 for the zero code and NaN codes,
+// which the saturating conversion never produces).
+__device__ __forceinline__ void fill_rcp_lut(float *lut) {
+    for (int i = threadIdx.x; i < 256; i += kThreads) {
+        const float v = e4m3_value(static_cast<uint32_t>(i));
+        lut[i] = (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
+    }
 }
 
-__device__ __forceinline__ uint32_t codes8(const float (&x)[8], float r) {
-    if (r == 0.0f) return 0u;  // scale 0: every code is 0 (+0)
-    return cvt_e2m1x8(__fmul_rn(x[0], r), __fmul_rn(x[1], r), __fmul_rn(x[2], r), __fmul_rn(x[3], r),
-                      __fmul_rn(x[4], r), __fmul_rn(x[5], r), __fmul_rn(x[6], r), __fmul_rn(x[7], r));
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Scale code of a block: E4M3_RN_sat(fp32(amax / 6)).
+__device__ __forceinline__ uint32_t scale_code(float amax) { return cvt_e4m3(__fdiv_rn(amax, 6.0f)); }
+
+// E2M1 codes of 16 values times r (fp32 products, rounded once each).
+__device__ __forceinline__ uint2 codes16(const uint64_t (&x2)[8], float r) {
+    if (r == 0.0f) return make_uint2(0u, 0u);  // scale 0: every code is 0 (+0)
+    const uint64_t rr = pack2(r, r);
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint64_t v = mul2(x2[i], rr);
+        y[2 * i] = lo2(v);
+        y[2 * i + 1] = hi2(v);
+    }
+    return make_uint2(cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]),
+                      cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]));
 }
 
-// One 128-token tile of Q or K (blocks of 16 along d).
+__device__ __forceinline__ float amax16(const uint64_t (&x2)[8]) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fmaxf(fabsf(lo2(x2[i])), fabsf(hi2(x2[i]))));
+    return a;
+}
+
+// ---------------------------------------------------------------- tiles
+// One staged 128-token tile of Q or K, quantized along d.  neg_mean: -mean
+// of K per channel (smoothing; negation is exact, so x + (-mean) is the
+// fp32 subtraction x - mean) or nullptr for Q.  Rows past N arrive as zeros
+// and get code 0 and scale 0.
 template <int D, bool kSmooth>
-__device__ __forceinline__ void qk_tile(const __nv_bfloat16 *__restrict__ src, int N, int tile,
-                                        const float *__restrict__ mean, uint8_t *__restrict__ codes,
-                                        uint8_t *__restrict__ sf) {
-    constexpr int kVec = D / 8;  // 16-byte vectors per row
-    constexpr int kIters = kTile * kVec / kThreads;
-    const int tid = threadIdx.x;
-    uint4 raw[kIters];
+__device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N, int tile,
+                                        const float *__restrict__ neg_mean, const float *__restrict__ rcp_lut,
+                                        uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+    constexpr int kBpt = D / 32;  // 16-element blocks per thread (4 or 2), consecutive along d
+    const int row = static_cast<int>(threadIdx.x) >> 1;
+    const int part = static_cast<int>(threadIdx.x) & 1;
+    const int t = tile * kTile + row;
+    uint32_t cw[2 * kBpt];
+    uint32_t scw = 0;
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-        const int hb = it * kThreads + tid;
-        const int t = tile * kTile + hb / kVec;
-        raw[it] = (t < N) ? ld_stream_v4(src + static_cast<size_t>(t) * D + (hb % kVec) * 8)
-                          : make_uint4(0u, 0u, 0u, 0u);
-    }
+    for (int i = 0; i < kBpt; ++i) {
+        const int ch0 = (part * kBpt + i) * 16;
+        const uint4 a = *reinterpret_cast<const uint4 *>(stage + tile_off(row, ch0));
+        const uint4 b = *reinterpret_cast<const uint4 *>(stage + tile_off(row, ch0 + 8));
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint64_t x2[8];
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-        const int hb = it * kThreads + tid;
-        const int row = hb / kVec;
-        const int v = hb % kVec;
-        const int t = tile * kTile + row;
-        float x[8];
-        bf16x8(raw[it], x);
+        for (int e = 0; e < 8; ++e) x2[e] = pack2(bf16_lo(w[e]), bf16_hi(w[e]));
         if (kSmooth && t < N) {
+            const float4 *nm = reinterpret_cast<const float4 *>(neg_mean + ch0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = __fsub_rn(x[i], mean[v * 8 + i]);
+            for (int e = 0; e < 4; ++e) {
+                const float4 m4 = nm[e];
+                x2[2 * e] = add2(x2[2 * e], pack2(m4.x, m4.y));
+                x2[2 * e + 1] = add2(x2[2 * e + 1], pack2(m4.z, m4.w));
+            }
         }
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        float r;
-        const uint32_t sc = block_scale(amax, r);
-        *reinterpret_cast<uint32_t *>(codes + static_cast<size_t>(t) * (D / 2) + v * 4) = codes8(x, r);
-        if ((v & 1) == 0) {
-            const int blk = v >> 1;
-            sf[(static_cast<size_t>(tile) * (D / 64) + (blk >> 2)) * 512 + atom_off(row, blk & 3)] =
-                static_cast<uint8_t>(sc);
-        }
+        const uint32_t sc = scale_code(amax16(x2));
+        const uint2 c = codes16(x2, rcp_lut[sc]);
+        cw[2 * i] = c.x;
+        cw[2 * i + 1] = c.y;
+        scw |= sc << (8 * i);
+    }
+    uint8_t *dst = codes + static_cast<size_t>(t) * (D / 2) + part * (kBpt * 8);
+    if constexpr (kBpt == 4) {
+        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        // blocks 4*part .. 4*part+3 are the four columns of atom `part`
+        *reinterpret_cast<uint32_t *>(sf + static_cast<size_t>(tile * 2 + part) * 512 + atom_off(row, 0)) = scw;
+    } else {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        // blocks 2*part, 2*part+1: columns 2*part, 2*part+1 of the tile's atom
+        *reinterpret_cast<uint16_t *>(sf + static_cast<size_t>(tile) * 512 + atom_off(row, 2 * part)) =
+            static_cast<uint16_t>(scw);
     }
 }
 
-// Quantize the 16 tokens (16*tb .. 16*tb+15 of this tile) of channel c.
+// One staged 128-token tile of V, quantized transposed: blocks of 16 tokens
+// per channel.  Thread: channel pair (2cp, 2cp+1), 16-token blocks
+// g*D/64 .. g*D/64 + D/64 - 1.
 template <int D>
-__device__ __forceinline__ void store_vblock(const float (&x)[16], int c, int tile, int tb, int Np,
-                                             uint8_t *__restrict__ vt, uint8_t *__restrict__ vsf) {
-    float amax = 0.0f;
+__device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int Np, int tile,
+                                       const float *__restrict__ rcp_lut, uint8_t *__restrict__ vt,
+                                       uint8_t *__restrict__ vsf) {
+    constexpr int kPairs = D / 2;
+    constexpr int kTbpt = D / 64;  // 16-token blocks per thread (2 or 1)
+    const int cp = static_cast<int>(threadIdx.x) % kPairs;
+    const int g = static_cast<int>(threadIdx.x) / kPairs;
+    uint32_t c0[2 * kTbpt], c1[2 * kTbpt];
+    uint32_t s0 = 0, s1 = 0;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
-    float r;
-    const uint32_t sc = block_scale(amax, r);
-    const float lo[8] = {x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]};
-    const float hi[8] = {x[8], x[9], x[10], x[11], x[12], x[13], x[14], x[15]};
-    uint2 w;
-    w.x = codes8(lo, r);
-    w.y = codes8(hi, r);
-    *reinterpret_cast<uint2 *>(vt + static_cast<size_t>(c) * (Np / 2) + tile * 64 + tb * 8) = w;
-    const size_t g = static_cast<size_t>(tile * 2 + (tb >> 2)) * 512;
-    vsf[g + 16 * (c & 31) + 4 * (c >> 5) + (tb & 3)] = static_cast<uint8_t>(sc);
-    if (D < 128) {  // padding channels of the 128-row scale atom
-        const int cz = c + D;
-        vsf[g + 16 * (cz & 31) + 4 * (cz >> 5) + (tb & 3)] = 0;
+    for (int i = 0; i < kTbpt; ++i) {
+        const int tb = g * kTbpt + i;
+        uint64_t x0[8], x1[8];
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+            const int r = tb * 16 + k;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(stage + tile_off(r, 2 * cp));
+            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(stage + tile_off(r + 1, 2 * cp));
+            x0[k / 2] = pack2(bf16_lo(w0), bf16_lo(w1));
+            x1[k / 2] = pack2(bf16_hi(w0), bf16_hi(w1));
+        }
+        const uint32_t sc0 = scale_code(amax16(x0));
+        const uint32_t sc1 = scale_code(amax16(x1));
+        const uint2 q0 = codes16(x0, rcp_lut[sc0]);
+        const uint2 q1 = codes16(x1, rcp_lut[sc1]);
+        c0[2 * i] = q0.x;
+        c0[2 * i + 1] = q0.y;
+        c1[2 * i] = q1.x;
+        c1[2 * i + 1] = q1.y;
+        s0 |= sc0 << (8 * i);
+        s1 |= sc1 << (8 * i);
+    }
+    const int c = 2 * cp;
+    uint8_t *row0 = vt + static_cast<size_t>(c) * (Np / 2) + tile * 64 + g * (kTbpt * 8);
+    uint8_t *row1 = row0 + Np / 2;
+    const int tb0 = g * kTbpt;
+    uint8_t *atom = vsf + static_cast<size_t>(tile * 2 + (tb0 >> 2)) * 512;
+    if constexpr (kTbpt == 2) {
+        *reinterpret_cast<uint4 *>(row0) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+        *reinterpret_cast<uint4 *>(row1) = make_uint4(c1[0], c1[1], c1[2], c1[3]);
+        *reinterpret_cast<uint16_t *>(atom + atom_off(c, tb0 & 3)) = static_cast<uint16_t>(s0);
+        *reinterpret_cast<uint16_t *>(atom + atom_off(c + 1, tb0 & 3)) = static_cast<uint16_t>(s1);
+    } else {
+        *reinterpret_cast<uint2 *>(row0) = make_uint2(c0[0], c0[1]);
+        *reinterpret_cast<uint2 *>(row1) = make_uint2(c1[0], c1[1]);
+        atom[atom_off(c, tb0 & 3)] = static_cast<uint8_t>(s0);
+        atom[atom_off(c + 1, tb0 & 3)] = static_cast<uint8_t>(s1);
+        // channels D .. 127 of the 128-row scale atom are padding (scale 0)
+        atom[atom_off(c + D, tb0 & 3)] = 0;
+        atom[atom_off(c + 1 + D, tb0 & 3)] = 0;
     }
 }
 
-// One 128-token tile of V, quantized transposed (blocks of 16 tokens per
-// channel).  stage: 128 x D bf16 in shared memory.
+// fp64 column sums of one staged K tile into this thread's accumulators:
+// channels 8v .. 8v+7 of rows r0, r0 + kRowStep, ...
 template <int D>
-__device__ __forceinline__ void v_tile(const __nv_bfloat16 *__restrict__ src, int N, int Np, int tile,
-                                       uint8_t *__restrict__ vt, uint8_t *__restrict__ vsf, uint32_t *stage) {
+__device__ __forceinline__ void ksum_tile(const uint8_t *__restrict__ stage, double (&acc)[8]) {
     constexpr int kVec = D / 8;
-    constexpr int kWords = D / 2;  // 32-bit words per staged row
-    constexpr int kIters = kTile * kVec / kThreads;
-    const int tid = threadIdx.x;
+    constexpr int kRowStep = kThreads / kVec;
+    const int v = static_cast<int>(threadIdx.x) % kVec;
+    const int r0 = static_cast<int>(threadIdx.x) / kVec;
 #pragma unroll
-    for (int it = 0; it < kIters; ++it) {
-        const int hb = it * kThreads + tid;
-        const int row = hb / kVec;
-        const int v = hb % kVec;
-        const int t = tile * kTile + row;
-        const uint4 val = (t < N) ? ld_stream_v4(src + static_cast<size_t>(t) * D + v * 8) : make_uint4(0u, 0u, 0u, 0u);
-        const int vs = v ^ ((row >> 4) & 7);
-        *reinterpret_cast<uint4 *>(stage + row * kWords + vs * 4) = val;
+    for (int r = r0; r < kTile; r += kRowStep) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(stage + tile_off(r, v * 8));
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += static_cast<double>(bf16_lo(u[e]));
+            acc[2 * e + 1] += static_cast<double>(bf16_hi(u[e]));
+        }
+    }
+}
+
+// Adds every thread's accumulators of the current chunk (warp shuffles over
+// the lanes holding the same channels, then the warps in order) and writes
+// the chunk's D sums; clears the accumulators.  Called by all threads.
+template <int D>
+__device__ __forceinline__ void ksum_flush(double (&acc)[8], double *red, double *__restrict__ out) {
+    constexpr int kVec = D / 8;
+    const int warp = static_cast<int>(threadIdx.x) >> 5;
+    const int lane = static_cast<int>(threadIdx.x) & 31;
+#pragma unroll
+    for (int off = kVec; off < 32; off <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+    }
+    if (lane < kVec) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp * D + lane * 8 + i] = acc[i];
     }
     __syncthreads();
-    constexpr int kUnits = (D / 2) * 8;  // (channel pair, 16-token block)
-    for (int u = tid; u < kUnits; u += kThreads) {
-        const int tb = u & 7;
-        const int cp = u >> 3;
-        float x0[16], x1[16];
+    for (int c = static_cast<int>(threadIdx.x); c < D; c += kThreads) {
+        double s = 0.0;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int row = tb * 16 + k;
-            const uint32_t w = stage[row * kWords + (((cp >> 2) ^ tb) << 2) + (cp & 3)];
-            x0[k] = __uint_as_float(w << 16);
-            x1[k] = __uint_as_float(w & 0xFFFF0000u);
+        for (int w = 0; w < kWarps; ++w) s += red[w * D + c];
+        out[c] = s;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+}
+
+// ------------------------------------------------------------- schedule
+// Work of the first launch for CTA g of G: a contiguous range of the Q and
+// V tiles (Q tiles of every (b, h) first, then V), then the K chunks
+// g, g+G, g+2G, ... one tile at a time.  The Q/V ranges are sized so that
+// every CTA ends up with about the same number of tiles: CTAs holding one
+// K chunk more (the first nK % G) take tpc fewer Q/V tiles.
+struct TileJob {
+    int kind;  // 0 = Q, 1 = V, 2 = K column sums
+    int bh;
+    int tile;
+    int chunk;      // K: chunk of the tile
+    bool last;      // K: last tile of its chunk
+};
+
+struct SchedA {
+    int ntile, nchunk, tpc, nqk;  // nqk = BH * ntile (Q tiles; V tiles follow)
+    int j, je;                    // Q/V tiles [j, je)
+    int ki, nK, G;                // next K chunk item, items, stride
+    int kbh, kch, kt, kt_end;     // current K chunk and its tiles [kt, kt_end)
+
+    __host__ __device__ void init(int BH, int ntile_, int nchunk_, int tpc_, int g, int G_) {
+        ntile = ntile_;
+        nchunk = nchunk_;
+        tpc = tpc_;
+        nqk = BH * ntile;
+        G = G_;
+        nK = BH * nchunk;
+        const int nqv = 2 * nqk;
+        const int a = nK / G, r = nK % G;
+        (void)a;
+        long long q_hi = (static_cast<long long>(nqv) + static_cast<long long>(r) * tpc + G - 1) / G;
+        long long q_lo = q_hi - tpc;
+        if (q_lo < 0) {
+            q_lo = 0;
+            q_hi = (nqv + (G - r) - 1) / (G - r);
         }
-        store_vblock<D>(x0, 2 * cp, tile, tb, Np, vt, vsf);
-        store_vblock<D>(x1, 2 * cp + 1, tile, tb, Np, vt, vsf);
+        const long long pre = g < r ? g * q_lo : r * q_lo + static_cast<long long>(g - r) * q_hi;
+        const long long cnt = g < r ? q_lo : q_hi;
+        j = static_cast<int>(pre < nqv ? pre : nqv);
+        je = static_cast<int>(pre + cnt < nqv ? pre + cnt : nqv);
+        ki = g;
+        kt = kt_end = 0;
+        kbh = kch = 0;
+    }
+    __host__ __device__ bool next(TileJob &t) {
+        if (j < je) {
+            const int kind = j < nqk ? 0 : 1;
+            const int jj = kind ? j - nqk : j;
+            t.kind = kind;
+            t.bh = jj / ntile;
+            t.tile = jj % ntile;
+            t.chunk = 0;
+            t.last = false;
+            ++j;
+            return true;
+        }
+        if (kt >= kt_end) {
+            if (ki >= nK) return false;
+            kbh = ki / nchunk;
+            kch = ki % nchunk;
+            kt = kch * tpc;
+            kt_end = kt + tpc < ntile ? kt + tpc : ntile;
+            ki += G;
+        }
+        t.kind = 2;
+        t.bh = kbh;
+        t.tile = kt;
+        t.chunk = kch;
+        t.last = kt + 1 == kt_end;
+        ++kt;
+        return true;
+    }
+};
+
+// ---------------------------------------------------------------- ring
+// kStages tile buffers, each filled by D/64 TMA boxes and one full barrier.
+template <int D>
+__device__ __forceinline__ void ring_issue(uint8_t *stage, uint64_t *full, const CUtensorMap *map, int bh,
+                                           int tile, uint64_t policy) {
+    mbar_arrive_expect_tx(full, QCfg<D>::kTileBytes);
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b)
+        tma_load_3d_hint(stage + b * QCfg<D>::kBoxBytes, map, b * kBoxCh, tile * kTile, bh, full, policy);
+}
+
+// Thread 0, after a failed wait: let every copy still in flight land
+// (bounded, ignoring the abort flag) before the CTA exits.
+__device__ __forceinline__ void ring_drain(uint64_t *full, int consumed, int issued) {
+    for (int m = consumed; m < issued; ++m) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(full + m % kStages, (m / kStages) & 1)) {
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                atomicOr(&g_sa3_status, 1u);
+                return;
+            }
+        }
     }
 }
 
-// fp64 partial sums of K over one 512-token chunk.
+struct SmemPtrs {
+    uint8_t *base;
+    uint64_t *full;
+    volatile int *abort;
+    float *lut;
+    double *red;
+    float *neg_mean;
+};
+
 template <int D>
-__device__ __forceinline__ void k_partial(const __nv_bfloat16 *__restrict__ src, int N, int chunk, int chunk_len,
-                                          double *__restrict__ part, double *red) {
-    constexpr int kVec = D / 8;
-    constexpr int kRows = kThreads / kVec;  // rows covered per step
-    const int tid = threadIdx.x;
-    const int v = tid % kVec;
-    const int r0 = tid / kVec;
+__device__ __forceinline__ SmemPtrs smem_setup(uint8_t *raw) {
+    using C = QCfg<D>;
+    const uint32_t a = smem_u32(raw);
+    SmemPtrs s;
+    s.base = raw + (((a + 1023u) & ~1023u) - a);
+    s.full = reinterpret_cast<uint64_t *>(s.base + C::oBar);
+    s.abort = reinterpret_cast<volatile int *>(s.full + kStages);
+    s.lut = reinterpret_cast<float *>(s.base + C::oLut);
+    s.red = reinterpret_cast<double *>(s.base + C::oRed);
+    s.neg_mean = reinterpret_cast<float *>(s.base + C::oMean);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(s.full + i, 1);
+        *s.abort = 0;
+        fence_mbar_init();
+    }
+    fill_rcp_lut(s.lut);
+    __syncthreads();
+    return s;
+}
+
+// -------------------------------------------------------------- kernels
+// First launch: Q and V tiles, then fp64 column sums of K per chunk.
+template <int D>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    quant_qvk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const QuantParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    pdl_trigger();  // the second launch may start once every CTA of this one has
+    const SmemPtrs sm = smem_setup<D>(smem_raw);
+    const int ntile = p.Np / kTile;
+    SchedA prod, cons;
+    prod.init(p.BH, ntile, p.nchunk, p.chunk / kTile, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
+    cons = prod;
+    const uint64_t pol_once = l2_policy_evict_first();
+    const uint64_t pol_k = l2_policy_evict_normal();
+    int issued = 0;
+    auto issue_next = [&](int s) {
+        TileJob t;
+        if (!prod.next(t)) return;
+        const CUtensorMap *m = t.kind == 0 ? &tm_q : (t.kind == 1 ? &tm_v : &tm_k);
+        ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, m, t.bh, t.tile, t.kind == 2 ? pol_k : pol_once);
+        ++issued;
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) issue_next(s);
+    }
     double acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-    const int t0 = chunk * chunk_len;
-    const int t1 = min(N, t0 + chunk_len);
-    constexpr int kBatch = 8;
-    for (int tb = t0 + r0; tb < t1; tb += kRows * kBatch) {
-        uint4 raw[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int t = tb + b * kRows;
-            raw[b] = (t < t1) ? ld_stream_v4(src + static_cast<size_t>(t) * D + v * 8) : make_uint4(0u, 0u, 0u, 0u);
+    int n = 0;
+    bool ok = true;
+    for (TileJob t; cons.next(t); ++n) {
+        const int s = n % kStages;
+        const bool got = mbar_wait(sm.full + s, (n / kStages) & 1, sm.abort);
+        if (__syncthreads_or(!got)) {
+            ok = false;
+            break;
         }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            float x[8];
-            bf16x8(raw[b], x);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(x[i]);
+        const uint8_t *st = sm.base + s * QCfg<D>::kTileBytes;
+        if (t.kind == 0) {
+            qk_tile<D, false>(st, p.N, t.tile, nullptr, sm.lut, p.q_fp4 + static_cast<size_t>(t.bh) * p.Np * (D / 2),
+                              p.q_sf + static_cast<size_t>(t.bh) * p.Np * (D / 16));
+        } else if (t.kind == 1) {
+            v_tile<D>(st, p.Np, t.tile, sm.lut, p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
+                      p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
+        } else {
+            ksum_tile<D>(st, acc);
+        }
+        __syncthreads();  // stage s has been read by every thread
+        if (t.kind == 2 && t.last)
+            ksum_flush<D>(acc, sm.red, p.part + (static_cast<size_t>(t.bh) * p.nchunk + t.chunk) * D);
+        if (threadIdx.x == 0) {
+            fence_proxy_async_smem();
+            issue_next(s);
         }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) red[r0 * D + v * 8 + i] = acc[i];
-    __syncthreads();
-    for (int c = tid; c < D; c += kThreads) {
-        double s = 0.0;
-        for (int r = 0; r < kRows; ++r) s += red[r * D + c];
-        part[static_cast<size_t>(chunk) * D + c] = s;
-    }
+    if (!ok && threadIdx.x == 0) ring_drain(sm.full, n, issued);
 }
 
+// Second launch: K tiles [g*T/G, (g+1)*T/G) of the T = BH * ntile tiles,
+// smoothed by the mean of their (b, h) and quantized.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 4) quant_qv_ksum_kernel(QuantParams p) {
-    __shared__ __align__(16) uint8_t smem[kTile * D * 2];
-    const int bh = blockIdx.y;
-    const int x = blockIdx.x;
-    const size_t in_off = static_cast<size_t>(bh) * p.N * D;
-    if (blockIdx.z == 0) {  // Q
-        qk_tile<D, false>(p.q + in_off, p.N, x, nullptr,
-                          p.q_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
-                          p.q_sf + static_cast<size_t>(bh) * p.Np * (D / 16));
-    } else if (blockIdx.z == 1) {  // V
-        v_tile<D>(p.v + in_off, p.N, p.Np, x, p.vt_fp4 + static_cast<size_t>(bh) * D * (p.Np / 2),
-                  p.vt_sf + static_cast<size_t>(bh) * p.Np * 8, reinterpret_cast<uint32_t *>(smem));
-    } else {  // K partial sums
-        if (x >= p.nchunk) return;
-        k_partial<D>(p.k + in_off, p.N, x, p.chunk, p.part + static_cast<size_t>(bh) * p.nchunk * D,
-                     reinterpret_cast<double *>(smem));
-    }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads) quant_k_kernel(QuantParams p) {
-    __shared__ float mean[D];
-    const int bh = blockIdx.y;
-    // mean of K over its N tokens: partial sums added in chunk order (fp64),
-    // one division, one rounding to fp32; tile 0 also stores it
-    for (int c = threadIdx.x; c < D; c += kThreads) {
-        const double *part = p.part + static_cast<size_t>(bh) * p.nchunk * D + c;
-        double s = 0.0;
-        for (int ch = 0; ch < p.nchunk; ++ch) s += part[static_cast<size_t>(ch) * D];
-        const float mu = __double2float_rn(s / static_cast<double>(p.N));
-        mean[c] = mu;
-        if (blockIdx.x == 0) p.k_mean[static_cast<size_t>(bh) * D + c] = mu;
-    }
-    __syncthreads();
-    qk_tile<D, true>(p.k + static_cast<size_t>(bh) * p.N * D, p.N, blockIdx.x, mean,
-                     p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
-                     p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16));
-}
-
-template <int D>
-cudaError_t launch_quant_d(const QuantParams &p, cudaStream_t stream) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    quant_k_kernel(const __grid_constant__ CUtensorMap tm_k, const QuantParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const SmemPtrs sm = smem_setup<D>(smem_raw);
     const int ntile = p.Np / kTile;
-    quant_qv_ksum_kernel<D><<<dim3(ntile, p.BH, 3), kThreads, 0, stream>>>(p);
-    quant_k_kernel<D><<<dim3(ntile, p.BH, 1), kThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    const long long T = static_cast<long long>(p.BH) * ntile;
+    const int i0 = static_cast<int>(T * blockIdx.x / gridDim.x);
+    const int i1 = static_cast<int>(T * (blockIdx.x + 1) / gridDim.x);
+    const uint64_t pol = l2_policy_evict_first();
+    int issued = 0;
+    // K is an input of this launch, not an output of the first one: its
+    // loads may start before the wait below
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages && i0 + s < i1; ++s, ++issued)
+            ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, &tm_k, (i0 + s) / ntile, (i0 + s) % ntile,
+                          pol);
+    }
+    pdl_wait();
+    int cur_bh = -1;
+    int n = 0;
+    bool ok = true;
+    for (; i0 + n < i1; ++n) {
+        const int idx = i0 + n;
+        const int bh = idx / ntile;
+        const int tile = idx % ntile;
+        if (bh != cur_bh) {
+            // mean of K over its N tokens: chunk sums added in chunk order
+            // (fp64), one division, one rounding to fp32; the CTA holding
+            // tile 0 of this (b, h) also stores it
+            for (int c = static_cast<int>(threadIdx.x); c < D; c += kThreads) {
+                const double *part = p.part + static_cast<size_t>(bh) * p.nchunk * D + c;
+                double v[kMaxChunks];
+#pragma unroll
+                for (int ch = 0; ch < kMaxChunks; ++ch) v[ch] = ch < p.nchunk ? part[static_cast<size_t>(ch) * D] : 0.0;
+                double s = 0.0;
+#pragma unroll
+                for (int ch = 0; ch < kMaxChunks; ++ch)
+                    if (ch < p.nchunk) s += v[ch];
+                const float mu = __double2float_rn(s / static_cast<double>(p.N));
+                sm.neg_mean[c] = -mu;
+                if (tile == 0) p.k_mean[static_cast<size_t>(bh) * D + c] = mu;
+            }
+            __syncthreads();
+            cur_bh = bh;
+        }
+        const int s = n % kStages;
+        const bool got = mbar_wait(sm.full + s, (n / kStages) & 1, sm.abort);
+        if (__syncthreads_or(!got)) {
+            ok = false;
+            break;
+        }
+        qk_tile<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean, sm.lut,
+                         p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
+                         p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16));
+        __syncthreads();  // stage s and neg_mean have been read by every thread
+        if (threadIdx.x == 0 && i0 + n + kStages < i1) {
+            fence_proxy_async_smem();
+            const int nx = i0 + n + kStages;
+            ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, &tm_k, nx / ntile, nx % ntile, pol);
+            ++issued;
+        }
+    }
+    if (!ok && threadIdx.x == 0) ring_drain(sm.full, n, issued);
 }
 
-}  // namespace
+template <int D>
+cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     cudaStream_t stream) {
+    using C = QCfg<D>;
+    if (p.nchunk > kMaxChunks || p.chunk % kTile != 0) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(quant_qvk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(quant_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const long long ntile = p.Np / kTile;
+    const long long work_a = 2 * p.BH * ntile + static_cast<long long>(p.BH) * p.nchunk;
+    const long long slots = static_cast<long long>(nsm) * kCtasPerSm;
+    const int grid_a = static_cast<int>(work_a < slots ? work_a : slots);
+    quant_qvk_kernel<D><<<grid_a, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long tiles_k = p.BH * ntile;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_k < slots ? tiles_k : slots));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quant_k_kernel<D>, tk, p);
+}
 
-inline cudaError_t launch_quant(const QuantParams &p, int d, cudaStream_t stream) {
-    return d == 128 ? launch_quant_d<128>(p, stream) : launch_quant_d<64>(p, stream);
+}  // namespace quant
+
+// Two launches: Q/V tiles and K chunk sums, then smoothed K tiles.  tq, tk,
+// tv: 3-D bf16 tensor maps {d, N, B*H} with 64 x 128 boxes and 128-byte
+// swizzle.
+inline cudaError_t launch_quant(const QuantParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                const CUtensorMap &tv, int d, cudaStream_t stream) {
+    return d == 128 ? quant::launch_d<128>(p, tq, tk, tv, stream) : quant::launch_d<64>(p, tq, tk, tv, stream);
 }
 
 }  // namespace sa3

@@ -54,6 +54,20 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, u
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [BH][N][d] as a 3-D tensor {d, N, BH}: boxes of 64 channels x 128
+// tokens x 1 head, 128-byte swizzle; tokens past N read as zeros.
+bool make_qkv_map(CUtensorMap *m, const void *base, int d, int N, int BH) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(int B, int H, int N, int d) {
@@ -126,9 +140,6 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, 
     const int64_t need = sa3_quant_workspace_bytes(B, H, N, d);
     if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
     sa3::QuantParams p;
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k = static_cast<const __nv_bfloat16 *>(k);
-    p.v = static_cast<const __nv_bfloat16 *>(v);
     p.q_fp4 = static_cast<uint8_t *>(out->q_fp4);
     p.q_sf = static_cast<uint8_t *>(out->q_sf);
     p.k_fp4 = static_cast<uint8_t *>(out->k_fp4);
@@ -142,7 +153,11 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, 
     p.Np = static_cast<int>(sa3_padded_len(N));
     p.chunk = static_cast<int>(sa3_kmean_chunk(N));
     p.nchunk = static_cast<int>(sa3_kmean_nchunk(N));
-    return sa3::launch_quant(p, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK : SA3_ERR_CUDA;
+    CUtensorMap tq, tk, tv;
+    if (!make_qkv_map(&tq, q, d, N, p.BH) || !make_qkv_map(&tk, k, d, N, p.BH) || !make_qkv_map(&tv, v, d, N, p.BH))
+        return SA3_ERR_CUDA;
+    return sa3::launch_quant(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK
+                                                                                                        : SA3_ERR_CUDA;
 }
 
 int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B, int H, int N, int d,

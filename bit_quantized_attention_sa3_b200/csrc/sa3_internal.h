@@ -9,10 +9,8 @@
 namespace sa3 {
 
 
+// Q, K and V themselves reach the quantizer as TMA tensor maps.
 struct QuantParams {
-    const __nv_bfloat16 *q;
-    const __nv_bfloat16 *k;
-    const __nv_bfloat16 *v;
     uint8_t *q_fp4;
     uint8_t *q_sf;
     uint8_t *k_fp4;
@@ -20,7 +18,7 @@ struct QuantParams {
     uint8_t *vt_fp4;
     uint8_t *vt_sf;
     float *k_mean;
-    double *part;  // [BH][nchunk][d] scratch
+    double *part;  // [BH][nchunk][d] scratch: fp64 column sums of K per chunk
     int BH;
     int N;
     int Np;
