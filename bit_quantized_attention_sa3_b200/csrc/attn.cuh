@@ -10,14 +10,15 @@
 //   O = alpha*O + P^ V^_j              block-scaled FP4 MMA, fp32 in TMEM
 // and finally out = bf16(O / l).
 //
-// One CTA = two 128-row Q tiles of one (b, h), 12 warps:
-//   warps 0-3  softmax for Q tile 0 (one thread per row = one TMEM lane)
-//   warps 4-7  softmax for Q tile 1
-//   warp  8    producer: TMA loads of Q, and of K / V^T codes + scales into
+// One CTA = two 128-row Q tiles of one (b, h), 18 warps:
+//   warps 0-7  softmax for Q tile 0: warp w owns TMEM lanes 32*(w%4) ..
+//              (one row per thread) and column half (w/4)%2, so each row
+//              is shared by two threads that exchange partial row maxima
+//   warps 8-15 softmax for Q tile 1
+//   warp 16    producer: TMA loads of Q, and of K / V^T codes + scales into
 //              a 3-stage ring (mbarrier transaction counts)
-//   warp  9    allocates TMEM and issues every tcgen05 op from one thread:
+//   warp 17    allocates TMEM and issues every tcgen05 op from one thread:
 //              scale-factor copies (tcgen05.cp), S = Q K^T, O += P V
-//   warps 10-11 idle (registers are granted per warpgroup)
 // TMEM (512 columns): S (128, shared by both tiles -- each softmax group
 // loads it to registers at once and releases it), O0, O1 (d each), and
 // the scale factors of Q0, Q1, K, P and V.  tcgen05.cp and tcgen05.mma
@@ -39,7 +40,12 @@ namespace attn {
 
 constexpr int kBlk = 128;
 constexpr int kStages = 3;
-constexpr int kThreads = 384;  // three warpgroups, 168 registers per thread
+constexpr int kSoftmaxWarps = 16;               // 2 tiles x 2 column halves x 4 lane quadrants
+constexpr int kWarpProducer = kSoftmaxWarps;     // warp 16
+constexpr int kWarpMma = kSoftmaxWarps + 1;      // warp 17
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;  // 576 threads, 112 registers each
+
+constexpr int kBarCountBytes = (17 + 2 * kStages) * 8;  // barrier slots below
 
 template <int D>
 struct Cfg {
@@ -69,7 +75,9 @@ struct Cfg {
     static constexpr int oPsf0 = oP1 + kPBytes;
     static constexpr int oPsf1 = oPsf0 + kPsfBytes;
     static constexpr int oLut = oPsf1 + kPsfBytes;     // 256 floats: 1 / E4M3 value
-    static constexpr int oBar = oLut + 1024;
+    static constexpr int oXch = oLut + 1024;           // row maxima [2 parity][2 tiles][2 halves][128]
+    static constexpr int oXl = oXch + 4096;            // row sums [2 tiles][2 halves][128]
+    static constexpr int oBar = oXl + 2048;
     static constexpr int kSmemBytes = oBar + 256 + 1024;
     // TMEM columns
     static constexpr uint32_t tS = 0;
@@ -82,6 +90,7 @@ struct Cfg {
     static constexpr uint32_t tSfv = tSfp + 8;
     static constexpr uint32_t kTmemCols = 512;
     static_assert(tSfv + 8 <= kTmemCols, "TMEM budget");
+    static_assert(kBarCountBytes + 8 <= 256, "barrier area");
 };
 
 // Barrier slots (uint64 each) after oBar.
@@ -94,8 +103,10 @@ enum : int {
     kBarPFull = 4 + 2 * kStages,     // 2
     kBarPvDone = 6 + 2 * kStages,    // 2
     kBarDrain = 8 + 2 * kStages,     // 1
-    kBarCount = 9 + 2 * kStages
+    kBarXch = 9 + 2 * kStages,       // 8: [tile][lane quadrant], 64 arrivals
+    kBarCount = 17 + 2 * kStages
 };
+static_assert(kBarCount * 8 == kBarCountBytes, "barrier slots");
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -178,12 +189,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(bars + kBarSFull + 0, 1);
         mbar_init(bars + kBarSFull + 1, 1);
-        mbar_init(bars + kBarSEmpty, 128);
-        mbar_init(bars + kBarPFull + 0, 128);
-        mbar_init(bars + kBarPFull + 1, 128);
+        mbar_init(bars + kBarSEmpty, 256);
+        mbar_init(bars + kBarPFull + 0, 256);
+        mbar_init(bars + kBarPFull + 1, 256);
         mbar_init(bars + kBarPvDone + 0, 1);
         mbar_init(bars + kBarPvDone + 1, 1);
         mbar_init(bars + kBarDrain, 1);
+        for (int x = 0; x < 8; ++x) mbar_init(bars + kBarXch + x, 64);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -193,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] =
             (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
     }
-    if (warp == 9) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -203,8 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const float *rcp_lut = reinterpret_cast<const float *>(base + C::oLut);
 
-    if (warp >= 8) {
-      if (warp == 8) {
+    if (warp >= kWarpProducer) {
+      if (warp == kWarpProducer) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
@@ -239,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
                 drain_wait(bars + kBarKvFull + j % kStages, (j / kStages) & 1);
         }
-    } else if (warp == 9) {
+    } else {
         // ----------------------------------------------------------- MMA
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_mxf4nvf4(128, 128);
@@ -327,17 +339,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else {
         // ------------------------------------------------------- softmax
-        const int i = warp >> 2;       // Q tile of this warpgroup
-        const int wq = warp & 3;       // TMEM sub-partition = rows 32*wq ..
-        const int r = wq * 32 + lane;  // row inside the tile
+        // Warp w: Q tile w/8, column half (w/4)%2 (64 of the 128 S columns,
+        // D/2 of the O columns), TMEM lanes 32*(w%4) .. : one row per thread,
+        // two threads per row.  The two halves of a row exchange their
+        // partial row maxima through shared memory (double-buffered by KV
+        // block parity), ordered by an mbarrier of 64 arrivals per pair of
+        // warps (bounded waits); each half keeps the row sum of its columns,
+        // added once at the end through the same barrier.
+        const int i = warp >> 3;         // Q tile of this warp
+        const int h = (warp >> 2) & 1;   // column half
+        const int wq = warp & 3;         // TMEM lane quadrant = rows 32*wq ..
+        const int r = wq * 32 + lane;    // row inside the tile
         const int tile = i ? tile1 : tile0;
         const int grow = tile * kBlk + r;
         const int n_i = i ? n1 : n0;
+        uint64_t *xbar = bars + kBarXch + 4 * i + wq;  // the two warps sharing these rows
         const float c2 = p.scale_log2;
         const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        const uint32_t tO = i ? C::tO1 : C::tO0;
+        const uint32_t tO = (i ? C::tO1 : C::tO0) + h * (D / 2);
         uint8_t *P = base + (i ? C::oP1 : C::oP0);
         uint8_t *Psf = base + (i ? C::oPsf1 : C::oPsf0);
+        float *xch = reinterpret_cast<float *>(base + C::oXch);  // [parity][tile][half][row]
+        float *xl = reinterpret_cast<float *>(base + C::oXl) + (i * 2) * kBlk;  // [tile][half][row]
         float m = -INFINITY;
         float l = 0.0f;
         bool ok = true;
@@ -347,33 +370,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t s[4][32];
+            uint32_t s[2][32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld32(trow + C::tS + 32 * q, s[q]);
+            for (int q = 0; q < 2; ++q) tmem_ld32(trow + C::tS + 64 * h + 32 * q, s[q]);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) reg_fence32(s[q]);
+            for (int q = 0; q < 2; ++q) reg_fence32(s[q]);
             tc_fence_before();
             mbar_arrive(bars + kBarSEmpty);
 
-            const int col0 = j * kBlk;
-            const bool tail = col0 + kBlk > p.N;
-            const bool diag = p.causal && (col0 + kBlk - 1 > tile * kBlk);
+            const int col0 = j * kBlk + 64 * h;
+            const bool tail = col0 + 64 > p.N;
+            const bool diag = p.causal && (col0 + 63 > tile * kBlk);
             if (tail || diag) {
                 // columns col0 + k with k >= lim are masked for this row
                 int lim = p.N - col0;
                 if (p.causal) lim = min(lim, grow - col0 + 1);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (32 * q + e >= lim) s[q][e] = __float_as_uint(-INFINITY);
                 }
             }
             // block maxima of the raw scores (c > 0, so max commutes with * c)
-            float bm[8];
+            float bm[4];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
+            for (int b = 0; b < 4; ++b) {
                 const uint32_t *x = &s[b >> 1][(b & 1) * 16];
                 const float m0 = max3f(__uint_as_float(x[0]), __uint_as_float(x[1]), __uint_as_float(x[2]));
                 const float m1 = max3f(__uint_as_float(x[3]), __uint_as_float(x[4]), __uint_as_float(x[5]));
@@ -382,37 +405,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m4 = max3f(__uint_as_float(x[12]), __uint_as_float(x[13]), __uint_as_float(x[14]));
                 bm[b] = max3f(max3f(m0, m1, m2), max3f(m3, m4, __uint_as_float(x[15])), m0);
             }
-            const float rmax = max3f(max3f(bm[0], bm[1], bm[2]), max3f(bm[3], bm[4], bm[5]), fmaxf(bm[6], bm[7]));
+            float *xs = xch + (((j & 1) * 2 + i) * 2) * kBlk;
+            xs[h * kBlk + r] = max3f(bm[0], bm[1], fmaxf(bm[2], bm[3]));
+            mbar_arrive(xbar);
+            if (!warp_wait(xbar, j & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const float rmax = fmaxf(xs[r], xs[kBlk + r]);
             const float m_new = fmaxf(m, __fmul_rn(rmax, c2));
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
             // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
             // two blocks per conversion; r_b = 1/s_b from the exact table
-            uint32_t scw[2];
-            float rb[8];
+            uint32_t scw;
+            float rb[4];
 #pragma unroll
-            for (int b = 0; b < 8; b += 2) {
+            for (int b = 0; b < 4; b += 2) {
                 const float a0 = ex2(__fsub_rn(__fmul_rn(bm[b], c2), m_new));
                 const float a1 = ex2(__fsub_rn(__fmul_rn(bm[b + 1], c2), m_new));
                 const uint32_t sc2 = cvt_e4m3x2(a1 * kSixth, a0 * kSixth);  // byte 0: block b
                 rb[b] = rcp_lut[sc2 & 0xFF];
                 rb[b + 1] = rcp_lut[sc2 >> 8];
-                if ((b & 2) == 0) scw[b >> 2] = sc2;
-                else scw[b >> 2] |= sc2 << 16;
+                if (b == 0) scw = sc2;
+                else scw |= sc2 << 16;
             }
             // P = 2^(t - m'), row sum of P (tree per block), codes of P * r
             const uint64_t cc = pack2(c2, c2);
             const uint64_t nn = pack2(nm, nm);
             uint64_t acc = pack2(0.0f, 0.0f);
-            uint32_t pc[16];
+            uint32_t pc[8];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) {
+            for (int b = 0; b < 4; ++b) {
                 const uint32_t *x = &s[b >> 1][(b & 1) * 16];
                 uint64_t vp[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1])), cc, nn);
-                    vp[i] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
+                for (int e = 0; e < 8; ++e) {
+                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), cc, nn);
+                    vp[e] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
                 }
                 const uint64_t s01 = add2(add2(vp[0], vp[1]), add2(vp[2], vp[3]));
                 const uint64_t s23 = add2(add2(vp[4], vp[5]), add2(vp[6], vp[7]));
@@ -420,14 +450,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t rr = pack2(rb[b], rb[b]);
                 uint64_t vy[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) vy[i] = mul2(vp[i], rr);
+                for (int e = 0; e < 8; ++e) vy[e] = mul2(vp[e], rr);
                 pc[2 * b] = cvt_e2m1x8(lo2(vy[0]), hi2(vy[0]), lo2(vy[1]), hi2(vy[1]), lo2(vy[2]), hi2(vy[2]),
                                        lo2(vy[3]), hi2(vy[3]));
                 pc[2 * b + 1] = cvt_e2m1x8(lo2(vy[4]), hi2(vy[4]), lo2(vy[5]), hi2(vy[5]), lo2(vy[6]), hi2(vy[6]),
                                            lo2(vy[7]), hi2(vy[7]));
             }
             const float sum = lo2(acc) + hi2(acc);
-            const uint32_t scw0 = scw[0], scw1 = scw[1];
             l = alpha * l + sum;
 
             // P buffer and O are free once the previous P V has completed.
@@ -439,24 +468,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
             }
             {
+                // this half's 32 code bytes = 16-byte chunks 2h, 2h+1 of the 64-byte row
                 uint8_t *prow = P + (r >> 3) * 512 + (r & 7) * 64;
                 const int sw = (r & 7) >> 1;
 #pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16)
-                    *reinterpret_cast<uint4 *>(prow + ((c16 ^ sw) << 4)) =
-                        make_uint4(pc[4 * c16], pc[4 * c16 + 1], pc[4 * c16 + 2], pc[4 * c16 + 3]);
-                *reinterpret_cast<uint32_t *>(Psf + 16 * (r & 31) + 4 * (r >> 5)) = scw0;
-                *reinterpret_cast<uint32_t *>(Psf + 512 + 16 * (r & 31) + 4 * (r >> 5)) = scw1;
+                for (int c = 0; c < 2; ++c)
+                    *reinterpret_cast<uint4 *>(prow + (((2 * h + c) ^ sw) << 4)) =
+                        make_uint4(pc[4 * c], pc[4 * c + 1], pc[4 * c + 2], pc[4 * c + 3]);
+                // blocks 4h .. 4h+3 = the four columns of scale atom h
+                *reinterpret_cast<uint32_t *>(Psf + 512 * h + 16 * (r & 31) + 4 * (r >> 5)) = scw;
             }
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-                // O = alpha * O for this warp's 32 rows
-                uint32_t o[D / 32][32];
+                // O = alpha * O for this warp's 32 rows, this half's D/2 columns
+                uint32_t o[D / 64][32];
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
+                for (int q = 0; q < D / 64; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
                 tmem_ld_wait();
                 const uint64_t aa = pack2(alpha, alpha);
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
+                for (int q = 0; q < D / 64; ++q) {
                     reg_fence32(o[q]);
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
@@ -473,12 +503,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(bars + kBarPFull + i);
             m = m_new;
         }
+        // row sum = the sums of the two halves, exchanged through the pair's
+        // barrier once more (phase n_i)
+        float l_row = 0.0f;
+        if (ok && n_i > 0) {
+            xl[h * kBlk + r] = l;
+            mbar_arrive(xbar);
+            ok = warp_wait(xbar, n_i & 1, abort_flag);
+            l_row = xl[r] + xl[kBlk + r];
+        }
         if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
             tc_fence_after();
-            const float inv = __frcp_rn(l);
-            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.N + grow) * D;
+            const float inv = __frcp_rn(l_row);
+            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.N + grow) * D + h * (D / 2);
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
+            for (int q = 0; q < D / 64; ++q) {
                 uint32_t o[32];
                 tmem_ld32(trow + tO + 32 * q, o);
                 tmem_ld_wait();
@@ -498,10 +537,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
