@@ -74,8 +74,8 @@ struct Cfg {
     static constexpr int oP1 = oP0 + kPBytes;
     static constexpr int oPsf0 = oP1 + kPBytes;
     static constexpr int oPsf1 = oPsf0 + kPsfBytes;
-    static constexpr int oLut = oPsf1 + kPsfBytes;     // 256 floats: 1 / E4M3 value
-    static constexpr int oXch = oLut + 1024;           // row maxima [2 parity][2 tiles][2 halves][128]
+    static constexpr int oLut = oPsf1 + kPsfBytes;     // 2 x 256 floats: log2(1/s), s per E4M3 code s
+    static constexpr int oXch = oLut + 2048;           // row maxima [2 parity][2 tiles][2 halves][128]
     static constexpr int oXl = oXch + 4096;            // row sums [2 tiles][2 halves][128]
     static constexpr int oBar = oXl + 2048;
     static constexpr int kSmemBytes = oBar + 256 + 1024;
@@ -200,10 +200,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
     }
     if (threadIdx.x < 256) {
-        // exact IEEE reciprocal of every E4M3 scale; 0 for scale 0 (and NaN codes)
+        // per E4M3 scale code: log2(1/s) and s.  Code 0 (and the NaN codes,
+        // which the saturating conversion never produces) map to log2 = 0,
+        // s = 1: such a block holds only P < 6 * 2^-10, whose codes at scale
+        // 1 are all 0, exactly as at scale 0, and whose row-sum terms stay P.
         const float v = e4m3_value(threadIdx.x);
-        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] =
-            (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
+        const bool unit = v == 0.0f || v != v;
+        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] = unit ? 0.0f : -log2f(v);
+        reinterpret_cast<float *>(base + C::oLut)[256 + threadIdx.x] = unit ? 1.0f : v;
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -213,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const float *rcp_lut = reinterpret_cast<const float *>(base + C::oLut);
+    const float *lg_lut = reinterpret_cast<const float *>(base + C::oLut);
+    const float *sv_lut = lg_lut + 256;
 
     if (warp >= kWarpProducer) {
       if (warp == kWarpProducer) {
@@ -417,46 +422,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
             // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
-            // two blocks per conversion; r_b = 1/s_b from the exact table
+            // two blocks per conversion
             uint32_t scw;
-            float rb[4];
+            float lg[4], sv[4];
 #pragma unroll
             for (int b = 0; b < 4; b += 2) {
                 const float a0 = ex2(__fsub_rn(__fmul_rn(bm[b], c2), m_new));
                 const float a1 = ex2(__fsub_rn(__fmul_rn(bm[b + 1], c2), m_new));
                 const uint32_t sc2 = cvt_e4m3x2(a1 * kSixth, a0 * kSixth);  // byte 0: block b
-                rb[b] = rcp_lut[sc2 & 0xFF];
-                rb[b + 1] = rcp_lut[sc2 >> 8];
+                lg[b] = lg_lut[sc2 & 0xFF];
+                lg[b + 1] = lg_lut[sc2 >> 8];
+                sv[b] = sv_lut[sc2 & 0xFF];
+                sv[b + 1] = sv_lut[sc2 >> 8];
                 if (b == 0) scw = sc2;
                 else scw |= sc2 << 16;
             }
-            // P = 2^(t - m'), row sum of P (tree per block), codes of P * r
+            // y = P / s_b = 2^(t - m' + log2(1/s_b)) (the 1/s_b folded into the
+            // exponent), codes of y; the row sum of P is sum_b s_b * sum(y)
             const uint64_t cc = pack2(c2, c2);
-            const uint64_t nn = pack2(nm, nm);
-            uint64_t acc = pack2(0.0f, 0.0f);
+            float sum = 0.0f;
             uint32_t pc[8];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const uint32_t *x = &s[b >> 1][(b & 1) * 16];
-                uint64_t vp[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), cc, nn);
-                    vp[e] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
-                }
-                const uint64_t s01 = add2(add2(vp[0], vp[1]), add2(vp[2], vp[3]));
-                const uint64_t s23 = add2(add2(vp[4], vp[5]), add2(vp[6], vp[7]));
-                acc = add2(acc, add2(s01, s23));
-                const uint64_t rr = pack2(rb[b], rb[b]);
+                const float bias = __fadd_rn(nm, lg[b]);
+                const uint64_t bb = pack2(bias, bias);
                 uint64_t vy[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) vy[e] = mul2(vp[e], rr);
+                for (int e = 0; e < 8; ++e) {
+                    const uint64_t t2 = fma2(pack2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1])), cc, bb);
+                    vy[e] = pack2(ex2(lo2(t2)), ex2(hi2(t2)));
+                }
+                const uint64_t s01 = add2(add2(vy[0], vy[1]), add2(vy[2], vy[3]));
+                const uint64_t s23 = add2(add2(vy[4], vy[5]), add2(vy[6], vy[7]));
+                const uint64_t sb = add2(s01, s23);
+                sum = fmaf(sv[b], lo2(sb) + hi2(sb), sum);
                 pc[2 * b] = cvt_e2m1x8(lo2(vy[0]), hi2(vy[0]), lo2(vy[1]), hi2(vy[1]), lo2(vy[2]), hi2(vy[2]),
                                        lo2(vy[3]), hi2(vy[3]));
                 pc[2 * b + 1] = cvt_e2m1x8(lo2(vy[4]), hi2(vy[4]), lo2(vy[5]), hi2(vy[5]), lo2(vy[6]), hi2(vy[6]),
                                            lo2(vy[7]), hi2(vy[7]));
             }
-            const float sum = lo2(acc) + hi2(acc);
             l = alpha * l + sum;
 
             // P buffer and O are free once the previous P V has completed.
