@@ -259,49 +259,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ----------------------------------------------------------- MMA
         if (lane == 0) {
+            // This thread shares its SM sub-partition with four busy softmax
+            // warps, so its instruction stream is kept short: shared-memory
+            // descriptors are built from precomputed low words (address >> 4
+            // | leading offset << 16) and a per-operand-kind high word, and
+            // ring positions advance incrementally.
             constexpr uint32_t idesc_qk = idesc_mxf4nvf4(128, 128);
             constexpr uint32_t idesc_pv = idesc_mxf4nvf4(128, D);
-            int nqk = 0;
-            auto stage_s = [&](int j) -> uint32_t {
-                return base_s + C::oStage + static_cast<uint32_t>(j % kStages) * C::kStageBytes;
+            constexpr uint32_t kHiQK = (static_cast<uint32_t>(C::kQKSbo) >> 4) | (1u << 14) | (C::kQKLayout << 29);
+            constexpr uint32_t kHiPV = (512u >> 4) | (1u << 14) | (4u << 29);
+            constexpr uint32_t kHiSF = (128u >> 4) | (1u << 14);
+            constexpr uint32_t kStageLo = static_cast<uint32_t>(C::kStageBytes) >> 4;
+            auto lo_of = [](uint32_t saddr, uint32_t lead) -> uint32_t {
+                return ((saddr >> 4) & 0x3FFFu) | (lead << 16);
             };
-            auto copy_ksf = [&](int j) {
+            auto desc = [](uint32_t lo, uint32_t hi) -> uint64_t {
+                uint64_t d;
+                asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+                return d;
+            };
+            const uint32_t st0 = base_s + C::oStage;
+            const uint32_t k_lo0 = lo_of(st0 + C::sK, 1), v_lo0 = lo_of(st0 + C::sV, 1);
+            const uint32_t ksf_lo0 = lo_of(st0 + C::sKsf, 8), vsf_lo0 = lo_of(st0 + C::sVsf, 8);
+            const uint32_t q_lo0 = lo_of(base_s + C::oQ0, 1), q_lo1 = lo_of(base_s + C::oQ1, 1);
+            const uint32_t p_lo0 = lo_of(base_s + C::oP0, 1), p_lo1 = lo_of(base_s + C::oP1, 1);
+            const uint32_t psf_lo0 = lo_of(base_s + C::oPsf0, 8), psf_lo1 = lo_of(base_s + C::oPsf1, 8);
+            const uint32_t t_s = tmem + C::tS, t_sfk = tmem + C::tSfk, t_sfp = tmem + C::tSfp, t_sfv = tmem + C::tSfv;
+            int nqk = 0;
+            auto copy_ksf = [&](int s) {
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a)
-                    tc_cp_32x128b_warpx4(tmem + C::tSfk + 4 * a, sdesc_sf_atom(stage_s(j) + C::sKsf + 512 * a));
+                    tc_cp_32x128b_warpx4(t_sfk + 4 * a, desc(ksf_lo0 + s * kStageLo + 32 * a, kHiSF));
             };
-            auto issue_qk = [&](int i, int j) -> bool {
+            auto issue_qk = [&](int i, int s) -> bool {
                 if (nqk > 0 && !mbar_wait(bars + kBarSEmpty, (nqk - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t qa = base_s + (i ? C::oQ1 : C::oQ0);
-                const uint32_t kb = stage_s(j) + C::sK;
+                const uint32_t qa = i ? q_lo1 : q_lo0;
+                const uint32_t kb = k_lo0 + s * kStageLo;
+                const uint32_t sfq = tmem + (i ? C::tSfq1 : C::tSfq0);
 #pragma unroll
                 for (int kc = 0; kc < D / 64; ++kc)
-                    tc_mma_mxf4nvf4(tmem + C::tS, sdesc_kmajor_sw(qa + 32 * kc, C::kQKSbo, C::kQKLayout),
-                                    sdesc_kmajor_sw(kb + 32 * kc, C::kQKSbo, C::kQKLayout), idesc_qk,
-                                    tmem + (i ? C::tSfq1 : C::tSfq0) + 4 * kc, tmem + C::tSfk + 4 * kc, kc > 0);
+                    tc_mma_mxf4nvf4(t_s, desc(qa + 2 * kc, kHiQK), desc(kb + 2 * kc, kHiQK), idesc_qk, sfq + 4 * kc,
+                                    t_sfk + 4 * kc, kc > 0);
                 tc_commit(bars + kBarSFull + i);
                 ++nqk;
                 return true;
             };
-            auto issue_pv = [&](int i, int j, bool load_vsf) -> bool {
+            auto issue_pv = [&](int i, int j, int s, bool load_vsf) -> bool {
                 if (!mbar_wait(bars + kBarPFull + i, j & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t pa = base_s + (i ? C::oP1 : C::oP0);
-                const uint32_t psf = base_s + (i ? C::oPsf1 : C::oPsf0);
-                const uint32_t vb = stage_s(j) + C::sV;
-                const uint32_t vsf = stage_s(j) + C::sVsf;
-                tc_cp_32x128b_warpx4(tmem + C::tSfp, sdesc_sf_atom(psf));
-                tc_cp_32x128b_warpx4(tmem + C::tSfp + 4, sdesc_sf_atom(psf + 512));
+                const uint32_t pa = i ? p_lo1 : p_lo0;
+                const uint32_t psf = i ? psf_lo1 : psf_lo0;
+                const uint32_t vb = v_lo0 + s * kStageLo;
+                tc_cp_32x128b_warpx4(t_sfp, desc(psf, kHiSF));
+                tc_cp_32x128b_warpx4(t_sfp + 4, desc(psf + 32, kHiSF));
                 if (load_vsf) {
-                    tc_cp_32x128b_warpx4(tmem + C::tSfv, sdesc_sf_atom(vsf));
-                    tc_cp_32x128b_warpx4(tmem + C::tSfv + 4, sdesc_sf_atom(vsf + 512));
+                    const uint32_t vsf = vsf_lo0 + s * kStageLo;
+                    tc_cp_32x128b_warpx4(t_sfv, desc(vsf, kHiSF));
+                    tc_cp_32x128b_warpx4(t_sfv + 4, desc(vsf + 32, kHiSF));
                 }
+                const uint32_t t_o = tmem + (i ? C::tO1 : C::tO0);
 #pragma unroll
                 for (int kc = 0; kc < 2; ++kc)
-                    tc_mma_mxf4nvf4(tmem + (i ? C::tO1 : C::tO0), sdesc_kmajor_sw(pa + 32 * kc, 512, 4u),
-                                    sdesc_kmajor_sw(vb + 32 * kc, 512, 4u), idesc_pv, tmem + C::tSfp + 4 * kc,
-                                    tmem + C::tSfv + 4 * kc, (j > 0 || kc > 0) ? 1u : 0u);
+                    tc_mma_mxf4nvf4(t_o, desc(pa + 2 * kc, kHiPV), desc(vb + 2 * kc, kHiPV), idesc_pv, t_sfp + 4 * kc,
+                                    t_sfv + 4 * kc, (j > 0 || kc > 0) ? 1u : 0u);
                 tc_commit(bars + kBarPvDone + i);
                 return true;
             };
@@ -323,18 +344,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (n0 > 0) ok = issue_qk(0, 0);
                 if (ok && n1 > 0) ok = issue_qk(1, 0);
             }
+            // s: ring stage of block j; s1, ph1: stage and parity of block j + 1
+            int s = 0, s1 = kStages > 1 ? 1 : 0;
+            uint32_t ph1 = kStages > 1 ? 0u : 1u;
             for (int j = 0; ok && j < nmax; ++j) {
                 if (j + 1 < nmax) {
-                    ok = mbar_wait(bars + kBarKvFull + (j + 1) % kStages, ((j + 1) / kStages) & 1, abort_flag);
+                    ok = mbar_wait(bars + kBarKvFull + s1, ph1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    copy_ksf(j + 1);
+                    copy_ksf(s1);
                 }
-                if (j + 1 < n0 && !(ok = issue_qk(0, j + 1))) break;
-                if (j < n0 && !(ok = issue_pv(0, j, true))) break;
-                if (j + 1 < n1 && !(ok = issue_qk(1, j + 1))) break;
-                if (j < n1 && !(ok = issue_pv(1, j, !(j < n0)))) break;
-                tc_commit(bars + kBarKvEmpty + j % kStages);
+                if (j + 1 < n0 && !(ok = issue_qk(0, s1))) break;
+                if (j < n0 && !(ok = issue_pv(0, j, s, true))) break;
+                if (j + 1 < n1 && !(ok = issue_qk(1, s1))) break;
+                if (j < n1 && !(ok = issue_pv(1, j, s, !(j < n0)))) break;
+                tc_commit(bars + kBarKvEmpty + s);
+                s = s1;
+                if (++s1 == kStages) {
+                    s1 = 0;
+                    ph1 ^= 1u;
+                }
             }
             // Every tcgen05 op issued above completes before TMEM is freed.
             tc_commit(bars + kBarDrain);
