@@ -72,11 +72,11 @@ def _load():
         lib.oracle_kmean.restype = None
         lib.oracle_kmean.argtypes = [P, I, I, I, I, P]
         lib.oracle_quantize_qkv.restype = None
-        lib.oracle_quantize_qkv.argtypes = [P, P, P, I, I, I, I, I] + [P] * 7
+        lib.oracle_quantize_qkv.argtypes = [P, P, P, I, I, I, I, I, I] + [P] * 7
         lib.oracle_attn_fwd.restype = None
-        lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, F, P, I, P]
+        lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, I, F, P, I, P]
         lib.oracle_attn_exact.restype = None
-        lib.oracle_attn_exact.argtypes = [P, P, P, I, I, I, I, I, F, P, P, I, P]
+        lib.oracle_attn_exact.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, I, P]
         lib.oracle_num_threads.restype = I
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -137,15 +137,19 @@ def kmean(k) -> np.ndarray:
 
 
 def quantize_qkv(q, k, v, smooth_k: bool = True) -> dict:
-    """Returns canonical-layout arrays: q_codes/k_codes [B,H,Np,d/2],
-    q_sf/k_sf [B,H,Np,d/16], vt_codes [B,H,d,Np/2], vt_sf [B,H,d,Np/16],
-    k_mean [B,H,d]."""
+    """Returns canonical-layout arrays: q_codes [B,H,Np(Nq),d/2], q_sf
+    [B,H,Np(Nq),d/16], k_codes/k_sf the same over Np(Nkv), vt_codes
+    [B,H,d,Np(Nkv)/2], vt_sf [B,H,d,Np(Nkv)/16], k_mean [B,H,d]; and the
+    lengths n_q, n_kv.  q is [B,H,Nq,d], k and v are [B,H,Nkv,d]."""
     q, k, v = _as_u16(q), _as_u16(k), _as_u16(v)
-    B, H, N, d = q.shape
+    B, H, Nq, d = q.shape
+    N = k.shape[2]
+    assert k.shape == v.shape and k.shape[:2] == (B, H) and k.shape[3] == d
+    Npq = padded_len(Nq)
     Np = padded_len(N)
     r = dict(
-        q_codes=np.zeros((B, H, Np, d // 2), np.uint8),
-        q_sf=np.zeros((B, H, Np, d // VEC), np.uint8),
+        q_codes=np.zeros((B, H, Npq, d // 2), np.uint8),
+        q_sf=np.zeros((B, H, Npq, d // VEC), np.uint8),
         k_codes=np.zeros((B, H, Np, d // 2), np.uint8),
         k_sf=np.zeros((B, H, Np, d // VEC), np.uint8),
         vt_codes=np.zeros((B, H, d, Np // 2), np.uint8),
@@ -153,9 +157,10 @@ def quantize_qkv(q, k, v, smooth_k: bool = True) -> dict:
         k_mean=np.zeros((B, H, d), np.float32),
     )
     _load().oracle_quantize_qkv(
-        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(bool(smooth_k)),
+        _ptr(q), _ptr(k), _ptr(v), B, H, Nq, N, d, int(bool(smooth_k)),
         _ptr(r["q_codes"]), _ptr(r["q_sf"]), _ptr(r["k_codes"]), _ptr(r["k_sf"]),
         _ptr(r["vt_codes"]), _ptr(r["vt_sf"]), _ptr(r["k_mean"]))
+    r["n_q"], r["n_kv"] = Nq, N
     return r
 
 
@@ -167,10 +172,14 @@ def _units_arr(units):
 
 
 def attn_fwd(qz: dict, N: int, causal: bool, sm_scale: float | None = None,
-             units=None, out: np.ndarray | None = None) -> np.ndarray:
-    """Tiled FP4 attention on canonical-layout quantized operands.
-    Returns bf16 bits uint16 [B,H,N,d]; rows outside ``units`` stay as in
-    ``out`` (zeros by default).  ``units`` lists (b*H+h, q_block) pairs."""
+             units=None, out: np.ndarray | None = None, n_kv: int | None = None) -> np.ndarray:
+    """Tiled FP4 attention on canonical-layout quantized operands with N
+    query rows and ``n_kv`` key columns (default: qz["n_kv"] if present,
+    else N).  Returns bf16 bits uint16 [B,H,N,d]; rows outside ``units``
+    stay as in ``out`` (zeros by default).  ``units`` lists (b*H+h,
+    q_block) pairs."""
+    if n_kv is None:
+        n_kv = qz.get("n_kv", N)
     B, H, Np, dh = qz["q_codes"].shape
     d = dh * 2
     if sm_scale is None:
@@ -180,24 +189,26 @@ def attn_fwd(qz: dict, N: int, causal: bool, sm_scale: float | None = None,
     u, nu = _units_arr(units)
     arrs = [np.ascontiguousarray(qz[n]) for n in
             ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf")]
-    _load().oracle_attn_fwd(*[_ptr(a) for a in arrs], B, H, N, d, int(bool(causal)),
+    _load().oracle_attn_fwd(*[_ptr(a) for a in arrs], B, H, N, n_kv, d, int(bool(causal)),
                             float(sm_scale), _ptr(u), nu, _ptr(out))
     return out
 
 
 def attn_exact(q, k, v, causal: bool, sm_scale: float | None = None,
                k_sub: np.ndarray | None = None, units=None) -> np.ndarray:
-    """fp64 softmax attention of the bf16 inputs; returns float64 [B,H,N,d]
-    (rows outside ``units`` are zero)."""
+    """fp64 softmax attention of the bf16 inputs (q [B,H,Nq,d], k and v
+    [B,H,Nkv,d]); returns float64 [B,H,Nq,d] (rows outside ``units`` are
+    zero)."""
     q, k, v = _as_u16(q), _as_u16(k), _as_u16(v)
     B, H, N, d = q.shape
+    Nkv = k.shape[2]
     if sm_scale is None:
         sm_scale = 1.0 / float(np.sqrt(d))
     out = np.zeros((B, H, N, d), np.float64)
     if k_sub is not None:
         k_sub = np.ascontiguousarray(k_sub, dtype=np.float32)
     u, nu = _units_arr(units)
-    _load().oracle_attn_exact(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, int(bool(causal)),
+    _load().oracle_attn_exact(_ptr(q), _ptr(k), _ptr(v), B, H, N, Nkv, d, int(bool(causal)),
                               float(sm_scale), _ptr(k_sub), _ptr(u), nu, _ptr(out))
     return out
 

@@ -29,8 +29,8 @@
  * contraction dimension (d for Q and K, tokens for V and P).
  *
  * Readings where the pages are silent (each is restated where it is used):
- *  R1 the K mean runs over the N real tokens of one (batch, head); summed in
- *     fp64 in token order, divided by N in fp64, rounded once to fp32;
+ *  R1 the K mean runs over the Nkv real tokens of one (batch, head); summed
+ *     in fp64 in token order, divided by Nkv in fp64, rounded once to fp32;
  *  R2 K_s = fp32(K) - mean, one fp32 subtraction;
  *  R3 block scale s = E4M3_RN_satfinite(fp32(amax / 6)); r = fp32(1 / s);
  *     code = E2M1_RN_satfinite(fp32(x * r)); s == 0 gives all-zero codes;
@@ -42,7 +42,12 @@
  *     c = fp32(sm_scale * log2(e)) in fp32 before the softmax, exp base 2;
  *  R8 P = exp2(t - m_new) with m_new the running max including the current
  *     block; the row sum l accumulates the unquantized P;
- *  R9 columns >= N and, when causal, columns > row are -inf before the max.
+ *  R9 columns >= Nkv and, when causal, columns > row + Nkv - Nq are -inf
+ *     before the max;
+ *  R11 Q may have fewer or more tokens (Nq) than K and V (Nkv); the causal
+ *     mask then aligns the last query with the last key (for Nq == Nkv this
+ *     is the usual lower-triangular mask);
+ *  R12 a query row that sees no key at all (causal, Nq > Nkv) outputs 0.
  */
 #include <math.h>
 #include <stdint.h>
@@ -199,28 +204,50 @@ void oracle_kmean(const uint16_t *k, int B, int H, int N, int d, float *mean)
 }
 
 /* ----------------------------------------------------- quantization (R1-R6)
- * Canonical layouts written here (N_p = N rounded up to 128):
- *   q_codes, k_codes : [B*H][N_p][d/2]   bytes
- *   q_sf, k_sf       : [B*H][N_p][d/16]  E4M3 bytes
- *   vt_codes         : [B*H][d][N_p/2]   bytes (V transposed)
- *   vt_sf            : [B*H][d][N_p/16]  E4M3 bytes
- *   k_mean           : [B*H][d] fp32
- * Padding tokens (t >= N) get code 0 and scale byte 0.
+ * Q has Nq tokens, K and V have Nkv (Nq == Nkv for self-attention).
+ * Canonical layouts written here (Np = a length rounded up to 128):
+ *   q_codes          : [B*H][Np(Nq)][d/2]    bytes
+ *   q_sf             : [B*H][Np(Nq)][d/16]   E4M3 bytes
+ *   k_codes, k_sf    : the same with Np(Nkv)
+ *   vt_codes         : [B*H][d][Np(Nkv)/2]   bytes (V transposed)
+ *   vt_sf            : [B*H][d][Np(Nkv)/16]  E4M3 bytes
+ *   k_mean           : [B*H][d] fp32, the mean over the Nkv tokens of K
+ * Padding tokens get code 0 and scale byte 0.
  * smooth_k = 0 skips the subtraction (used to measure what smoothing buys). */
+static void quant_rows(const uint16_t *x_in, long bh, int N, int Np, int d, const float *sub,
+                       uint8_t *codes_out, uint8_t *sf_out)
+{
+    float x[VEC];
+    int codes[VEC];
+    for (int t = 0; t < N; ++t) {
+        for (int b = 0; b < d / VEC; ++b) {
+            for (int i = 0; i < VEC; ++i) {
+                float xv = bf16_to_f32(x_in[(bh * N + t) * d + b * VEC + i]);
+                x[i] = sub ? xv - sub[b * VEC + i] : xv;  /* one fp32 subtraction (R2) */
+            }
+            int sc = quant_block(x, codes);
+            sf_out[(bh * Np + t) * (d / VEC) + b] = (uint8_t)sc;
+            for (int i = 0; i < VEC; i += 2)
+                codes_out[(bh * Np + t) * (d / 2) + (b * VEC + i) / 2] = (uint8_t)(codes[i] | (codes[i + 1] << 4));
+        }
+    }
+}
+
 void oracle_quantize_qkv(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                         int B, int H, int N, int d, int smooth_k,
+                         int B, int H, int Nq, int Nkv, int d, int smooth_k,
                          uint8_t *q_codes, uint8_t *q_sf,
                          uint8_t *k_codes, uint8_t *k_sf,
                          uint8_t *vt_codes, uint8_t *vt_sf, float *k_mean)
 {
     tables_init();
     const long BH = (long)B * H;
-    const int Np = oracle_padded_len(N);
-    oracle_kmean(k, B, H, N, d, k_mean);
+    const int Npq = oracle_padded_len(Nq);
+    const int Np = oracle_padded_len(Nkv);
+    oracle_kmean(k, B, H, Nkv, d, k_mean);
 
-    memset(q_codes, 0, (size_t)BH * Np * d / 2);
+    memset(q_codes, 0, (size_t)BH * Npq * d / 2);
+    memset(q_sf, 0, (size_t)BH * Npq * d / VEC);
     memset(k_codes, 0, (size_t)BH * Np * d / 2);
-    memset(q_sf, 0, (size_t)BH * Np * d / VEC);
     memset(k_sf, 0, (size_t)BH * Np * d / VEC);
     memset(vt_codes, 0, (size_t)BH * d * Np / 2);
     memset(vt_sf, 0, (size_t)BH * d * Np / VEC);
@@ -229,35 +256,15 @@ void oracle_quantize_qkv(const uint16_t *q, const uint16_t *k, const uint16_t *v
     for (long bh = 0; bh < BH; ++bh) {
         float x[VEC];
         int codes[VEC];
-        /* Q and K: blocks of 16 along d, per token. */
-        for (int t = 0; t < N; ++t) {
-            for (int b = 0; b < d / VEC; ++b) {
-                /* Q */
-                for (int i = 0; i < VEC; ++i)
-                    x[i] = bf16_to_f32(q[(bh * N + t) * d + b * VEC + i]);
-                int sc = quant_block(x, codes);
-                q_sf[(bh * Np + t) * (d / VEC) + b] = (uint8_t)sc;
-                for (int i = 0; i < VEC; i += 2)
-                    q_codes[(bh * Np + t) * (d / 2) + (b * VEC + i) / 2] =
-                        (uint8_t)(codes[i] | (codes[i + 1] << 4));
-                /* K, smoothed (R2) */
-                for (int i = 0; i < VEC; ++i) {
-                    float kv = bf16_to_f32(k[(bh * N + t) * d + b * VEC + i]);
-                    x[i] = smooth_k ? kv - k_mean[bh * d + b * VEC + i] : kv;
-                }
-                sc = quant_block(x, codes);
-                k_sf[(bh * Np + t) * (d / VEC) + b] = (uint8_t)sc;
-                for (int i = 0; i < VEC; i += 2)
-                    k_codes[(bh * Np + t) * (d / 2) + (b * VEC + i) / 2] =
-                        (uint8_t)(codes[i] | (codes[i + 1] << 4));
-            }
-        }
+        /* Q and K: blocks of 16 along d, per token; K smoothed (R2). */
+        quant_rows(q, bh, Nq, Npq, d, NULL, q_codes, q_sf);
+        quant_rows(k, bh, Nkv, Np, d, smooth_k ? k_mean + bh * d : NULL, k_codes, k_sf);
         /* V: blocks of 16 tokens, per channel (R6). */
         for (int c = 0; c < d; ++c) {
             for (int tb = 0; tb < Np / VEC; ++tb) {
                 for (int i = 0; i < VEC; ++i) {
                     int t = tb * VEC + i;
-                    x[i] = (t < N) ? bf16_to_f32(v[(bh * N + t) * d + c]) : 0.0f;
+                    x[i] = (t < Nkv) ? bf16_to_f32(v[(bh * Nkv + t) * d + c]) : 0.0f;
                 }
                 int sc = quant_block(x, codes);
                 vt_sf[(bh * d + c) * (Np / VEC) + tb] = (uint8_t)sc;
@@ -278,18 +285,23 @@ static double deq(const uint8_t *codes, const uint8_t *sf, long elem, long sf_id
 }
 
 /* ------------------------------------------------- tiled attention (R7-R9)
+ * Nq query rows, Nkv key/value columns.  causal masks col > row + Nkv - Nq
+ * (the last query row aligned with the last key, R11); a row that sees no
+ * column at all gets output 0 (R12).
  * units: n_units pairs (bh, q_block); NULL means every (bh, q_block).
- * out: bf16 [B*H][N][d]; only rows of the listed units are written. */
+ * out: bf16 [B*H][Nq][d]; only rows of the listed units are written. */
 void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                      const uint8_t *k_codes, const uint8_t *k_sf,
                      const uint8_t *vt_codes, const uint8_t *vt_sf,
-                     int B, int H, int N, int d, int causal, float sm_scale,
+                     int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
                      const int32_t *units, int n_units, uint16_t *out)
 {
     tables_init();
     const long BH = (long)B * H;
-    const int Np = oracle_padded_len(N);
-    const int nqb = Np / BLK;
+    const int Npq = oracle_padded_len(Nq);
+    const int Np = oracle_padded_len(Nkv);
+    const int nqb = Npq / BLK;
+    const int off = Nkv - Nq;
     const float c_log2 = (float)((double)sm_scale * 1.4426950408889634);
     const long total = units ? n_units : BH * nqb;
 
@@ -297,13 +309,19 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
     for (long u = 0; u < total; ++u) {
         long bh = units ? units[2 * u] : u / nqb;
         int qb = units ? units[2 * u + 1] : (int)(u % nqb);
-        int nkv = causal ? qb + 1 : Np / BLK;
+        /* KV blocks up to the last column any row of this Q block sees */
+        int nkv = Np / BLK;
+        if (causal) {
+            int last = qb * BLK + BLK - 1 + off;
+            int nb = last < 0 ? 0 : last / BLK + 1;
+            if (nb < nkv) nkv = nb;
+        }
         int ncol = nkv * BLK;
         /* Dequantized operands of this (batch, head), cached so that each
          * value is decoded once; the sums below are unchanged by this. */
         double *qrow = (double *)malloc(sizeof(double) * d);
-        double *khat = (double *)malloc(sizeof(double) * (size_t)ncol * d);
-        double *vhat = (double *)malloc(sizeof(double) * (size_t)ncol * d);
+        double *khat = (double *)malloc(sizeof(double) * ((size_t)ncol * d + 1));
+        double *vhat = (double *)malloc(sizeof(double) * ((size_t)ncol * d + 1));
         float *O = (float *)malloc(sizeof(float) * d);
         float t[BLK], p[BLK], phat[BLK];
         int codes[VEC];
@@ -316,10 +334,10 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                 vhat[(size_t)c * ncol + col] = deq(vt_codes, vt_sf, (bh * d + c) * Np + col,
                                                    (bh * d + c) * (Np / VEC) + col / VEC);
 
-        for (int row = qb * BLK; row < qb * BLK + BLK && row < N; ++row) {
+        for (int row = qb * BLK; row < qb * BLK + BLK && row < Nq; ++row) {
             for (int c = 0; c < d; ++c)
-                qrow[c] = deq(q_codes, q_sf, (bh * Np + row) * d + c,
-                              (bh * Np + row) * (d / VEC) + c / VEC);
+                qrow[c] = deq(q_codes, q_sf, (bh * Npq + row) * d + c,
+                              (bh * Npq + row) * (d / VEC) + c / VEC);
             float m = -INFINITY, l = 0.0f;
             for (int c = 0; c < d; ++c) O[c] = 0.0f;
 
@@ -328,7 +346,7 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                 float bmax = -INFINITY;
                 for (int i = 0; i < BLK; ++i) {
                     int col = j * BLK + i;
-                    if (col >= N || (causal && col > row)) { t[i] = -INFINITY; continue; }
+                    if (col >= Nkv || (causal && col > row + off)) { t[i] = -INFINITY; continue; }
                     double acc = 0.0;
                     for (int c = 0; c < d; ++c)
                         acc += qrow[c] * khat[(size_t)col * d + c];
@@ -366,7 +384,7 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                 m = m_new;
             }
             for (int c = 0; c < d; ++c)
-                out[(bh * N + row) * d + c] = oracle_f32_to_bf16(O[c] / l);
+                out[(bh * Nq + row) * d + c] = l > 0.0f ? oracle_f32_to_bf16(O[c] / l) : 0;
         }
         free(qrow);
         free(khat);
@@ -376,32 +394,39 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
 }
 
 /* --------------------------------------------- exact attention (fp64)
- * softmax(Q K^T * sm_scale) V on the bf16 inputs, no quantization.  k_sub,
- * if not NULL, is subtracted from K first (fp32 [B*H][d]); this is how the
- * smoothing invariance is checked.  Rows of the listed units only. */
+ * softmax(Q K^T * sm_scale) V on the bf16 inputs, no quantization, with the
+ * masks of oracle_attn_fwd.  k_sub, if not NULL, is subtracted from K first
+ * (fp32 [B*H][d]); this is how the smoothing invariance is checked.  Rows
+ * of the listed units only; a row that sees no column gets 0. */
 void oracle_attn_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                       int B, int H, int N, int d, int causal, float sm_scale,
+                       int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
                        const float *k_sub, const int32_t *units, int n_units,
                        double *out)
 {
     const long BH = (long)B * H;
-    const int nqb = oracle_padded_len(N) / BLK;
+    const int nqb = oracle_padded_len(Nq) / BLK;
+    const int off = Nkv - Nq;
     const long total = units ? n_units : BH * nqb;
 
 #pragma omp parallel for schedule(dynamic)
     for (long u = 0; u < total; ++u) {
         long bh = units ? units[2 * u] : u / nqb;
         int qb = units ? units[2 * u + 1] : (int)(u % nqb);
-        double *logit = (double *)malloc(sizeof(double) * N);
-        for (int row = qb * BLK; row < qb * BLK + BLK && row < N; ++row) {
-            int ncol = causal ? row + 1 : N;
+        double *logit = (double *)malloc(sizeof(double) * (Nkv + 1));
+        for (int row = qb * BLK; row < qb * BLK + BLK && row < Nq; ++row) {
+            int ncol = causal ? row + off + 1 : Nkv;
+            if (ncol > Nkv) ncol = Nkv;
+            if (ncol <= 0) {
+                for (int c = 0; c < d; ++c) out[(bh * Nq + row) * d + c] = 0.0;
+                continue;
+            }
             double mx = -INFINITY;
             for (int col = 0; col < ncol; ++col) {
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c) {
-                    double kk = bf16_to_f32(k[(bh * N + col) * d + c]);
+                    double kk = bf16_to_f32(k[(bh * Nkv + col) * d + c]);
                     if (k_sub) kk -= (double)k_sub[bh * d + c];
-                    acc += (double)bf16_to_f32(q[(bh * N + row) * d + c]) * kk;
+                    acc += (double)bf16_to_f32(q[(bh * Nq + row) * d + c]) * kk;
                 }
                 logit[col] = acc * (double)sm_scale;
                 if (logit[col] > mx) mx = logit[col];
@@ -414,8 +439,8 @@ void oracle_attn_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             for (int c = 0; c < d; ++c) {
                 double acc = 0.0;
                 for (int col = 0; col < ncol; ++col)
-                    acc += logit[col] * (double)bf16_to_f32(v[(bh * N + col) * d + c]);
-                out[(bh * N + row) * d + c] = acc / den;
+                    acc += logit[col] * (double)bf16_to_f32(v[(bh * Nkv + col) * d + c]);
+                out[(bh * Nq + row) * d + c] = acc / den;
             }
         }
         free(logit);
