@@ -65,6 +65,10 @@ def lib() -> ctypes.CDLL:
             L.sa3_quantize_qkv.argtypes = [P, P, P, I, I, I, I, ctypes.POINTER(_QKV), P, ctypes.c_size_t, P]
             L.sa3_attn_fwd.restype = I
             L.sa3_attn_fwd.argtypes = [ctypes.POINTER(_QKV), I, I, I, I, I, F, P, P]
+            L.sa3_quantize_qkv_lens.restype = I
+            L.sa3_quantize_qkv_lens.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(_QKV), P, ctypes.c_size_t, P]
+            L.sa3_attn_fwd_lens.restype = I
+            L.sa3_attn_fwd_lens.argtypes = [ctypes.POINTER(_QKV), I, I, I, I, I, I, F, P, P]
             L.sa3_device_status.restype = I
             L.sa3_device_status.argtypes = [P]
             _lib = L
@@ -92,8 +96,9 @@ def quant_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 @dataclasses.dataclass
 class QuantizedQKV:
-    """Device buffers of the quantized operands (layouts: include/sa3.h)."""
-    q_fp4: torch.Tensor   # u8 [B,H,Np,d/2]
+    """Device buffers of the quantized operands (layouts: include/sa3.h).
+    N is the key/value length; Nq the query length (None: equal to N)."""
+    q_fp4: torch.Tensor   # u8 [B,H,Np(Nq),d/2]
     q_sf: torch.Tensor    # u8, 128x4 scale atoms
     k_fp4: torch.Tensor   # u8 [B,H,Np,d/2]
     k_sf: torch.Tensor
@@ -104,6 +109,11 @@ class QuantizedQKV:
     H: int
     N: int
     d: int
+    Nq: int | None = None
+
+    @property
+    def n_q(self) -> int:
+        return self.N if self.Nq is None else self.Nq
 
     def struct(self) -> _QKV:
         return _QKV(self.q_fp4.data_ptr(), self.q_sf.data_ptr(), self.k_fp4.data_ptr(),
@@ -111,14 +121,17 @@ class QuantizedQKV:
                     self.k_mean.data_ptr())
 
 
-def empty_quantized(B: int, H: int, N: int, d: int, device="cuda") -> QuantizedQKV:
+def empty_quantized(B: int, H: int, N: int, d: int, device="cuda", Nq: int | None = None) -> QuantizedQKV:
+    """Buffers for keys/values of length N and queries of length Nq (default N)."""
     Np = padded_len(N)
+    Npq = padded_len(N if Nq is None else Nq)
     u8 = dict(dtype=torch.uint8, device=device)
     return QuantizedQKV(
-        q_fp4=torch.empty((B, H, Np, d // 2), **u8), q_sf=torch.empty(B * H * Np * d // 16, **u8),
+        q_fp4=torch.empty((B, H, Npq, d // 2), **u8), q_sf=torch.empty(B * H * Npq * d // 16, **u8),
         k_fp4=torch.empty((B, H, Np, d // 2), **u8), k_sf=torch.empty(B * H * Np * d // 16, **u8),
         vt_fp4=torch.empty((B, H, d, Np // 2), **u8), vt_sf=torch.empty(B * H * Np * 8, **u8),
-        k_mean=torch.empty((B, H, d), dtype=torch.float32, device=device), B=B, H=H, N=N, d=d)
+        k_mean=torch.empty((B, H, d), dtype=torch.float32, device=device), B=B, H=H, N=N, d=d,
+        Nq=None if Nq is None or Nq == N else Nq)
 
 
 def _stream_ptr(stream) -> int:
@@ -135,20 +148,30 @@ def _check_input(t: torch.Tensor, name: str):
 def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  out: QuantizedQKV | None = None, workspace: torch.Tensor | None = None,
                  stream=None) -> QuantizedQKV:
-    """sa3_quantize_qkv: K smoothing, then E2M1 codes + E4M3 scales of Q, K, V."""
+    """sa3_quantize_qkv: K smoothing, then E2M1 codes + E4M3 scales of Q, K, V.
+    q is [B,H,Nq,d]; k and v are [B,H,N,d] (N may differ from Nq:
+    sa3_quantize_qkv_lens)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_input(t, n)
-    if not (q.shape == k.shape == v.shape):
-        raise ValueError("q, k, v must have the same shape (self-attention)")
-    B, H, N, d = q.shape
+    if not (k.shape == v.shape and q.shape[:2] == k.shape[:2] and q.shape[3] == k.shape[3]):
+        raise ValueError("q must be [B,H,Nq,d] and k, v [B,H,N,d]")
+    B, H, Nq, d = q.shape
+    N = k.shape[2]
     if out is None:
-        out = empty_quantized(B, H, N, d, q.device)
+        out = empty_quantized(B, H, N, d, q.device, Nq=Nq)
+    if out.n_q != Nq or out.N != N:
+        raise ValueError("out was sized for other lengths")
     nbytes = quant_workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     st = out.struct()
-    rc = lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(st),
-                                workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if Nq == N:
+        rc = lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(st),
+                                    workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    else:
+        rc = lib().sa3_quantize_qkv_lens(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, Nq, N, d,
+                                         ctypes.byref(st), workspace.data_ptr(), workspace.numel(),
+                                         _stream_ptr(stream))
     if rc != SA3_OK:
         raise Sa3Error(rc, "sa3_quantize_qkv")
     return out
@@ -156,15 +179,21 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 def attn_fwd(qz: QuantizedQKV, causal: bool = False, sm_scale: float | None = None,
              out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """sa3_attn_fwd: FP4 attention of quantized operands; bf16 [B,H,N,d]."""
-    B, H, N, d = qz.B, qz.H, qz.N, qz.d
+    """sa3_attn_fwd: FP4 attention of quantized operands; bf16 [B,H,Nq,d].
+    With Nq != N (sa3_attn_fwd_lens) the causal mask aligns the last query
+    with the last key; a row that sees no key is 0."""
+    B, H, N, d, Nq = qz.B, qz.H, qz.N, qz.d, qz.n_q
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=qz.q_fp4.device)
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=qz.q_fp4.device)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     st = qz.struct()
-    rc = lib().sa3_attn_fwd(ctypes.byref(st), B, H, N, d, int(bool(causal)), float(sm_scale),
-                            out.data_ptr(), _stream_ptr(stream))
+    if Nq == N:
+        rc = lib().sa3_attn_fwd(ctypes.byref(st), B, H, N, d, int(bool(causal)), float(sm_scale),
+                                out.data_ptr(), _stream_ptr(stream))
+    else:
+        rc = lib().sa3_attn_fwd_lens(ctypes.byref(st), B, H, Nq, N, d, int(bool(causal)), float(sm_scale),
+                                     out.data_ptr(), _stream_ptr(stream))
     if rc != SA3_OK:
         raise Sa3Error(rc, "sa3_attn_fwd")
     return out

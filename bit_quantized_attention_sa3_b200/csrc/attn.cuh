@@ -166,7 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Q tiles, ordered by rank (heaviest pairs first when causal) and then
     // head; the pairs after them are split into single-tile units that fill
     // what would otherwise be a short last wave.
-    const int nqt = p.Np / kBlk;
+    const int nqt = p.Npq / kBlk;   // Q tiles
+    const int nkvt = p.Np / kBlk;   // KV blocks
+    const int off = p.N - p.Nq;     // causal: row r sees keys 0 .. r + off
     const int u = static_cast<int>(blockIdx.x);
     const bool single = u >= p.pair_units;
     const int pu = single ? p.pair_units + (u - p.pair_units) / 2 : u;
@@ -177,8 +179,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tile1 = tile0 + 1;
     if (tile0 >= nqt) return;  // second half of a split pair whose head has an odd tile count
     const bool valid1 = !single && tile1 < nqt;
-    const int n0 = p.causal ? tile0 + 1 : nqt;
-    const int n1 = valid1 ? (p.causal ? tile1 + 1 : nqt) : 0;
+    // KV blocks up to the last key any row of the tile sees (0: none)
+    auto n_blocks = [&](int tile) -> int {
+        if (!p.causal) return nkvt;
+        const int last = tile * kBlk + kBlk - 1 + off;
+        const int nb = last < 0 ? 0 : last / kBlk + 1;
+        return nb < nkvt ? nb : nkvt;
+    };
+    const int n0 = n_blocks(tile0);
+    const int n1 = valid1 ? n_blocks(tile1) : 0;
     const int nmax = n0 > n1 ? n0 : n1;
 
     if (threadIdx.x == 0) {
@@ -229,10 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tm_v);
             uint64_t *bq = bars + kBarQ;
             mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * (C::kQBytes + C::kSfBytes));
-            tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Np + tile0 * kBlk, bq);
+            tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Npq + tile0 * kBlk, bq);
             bulk_load(base + C::oQsf0, p.q_sf + static_cast<size_t>(bh * nqt + tile0) * C::kSfBytes, C::kSfBytes, bq);
             if (valid1) {
-                tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Np + tile1 * kBlk, bq);
+                tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Npq + tile1 * kBlk, bq);
                 bulk_load(base + C::oQsf1, p.q_sf + static_cast<size_t>(bh * nqt + tile1) * C::kSfBytes, C::kSfBytes,
                           bq);
             }
@@ -245,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint64_t *bf = bars + kBarKvFull + s;
                 mbar_arrive_expect_tx(bf, C::kQBytes + C::kSfBytes + C::kVBytes + C::kVsfBytes);
                 tma_load_2d(st + C::sK, &tm_k, 0, bh * p.Np + j * kBlk, bf);
-                bulk_load(st + C::sKsf, p.k_sf + static_cast<size_t>(bh * nqt + j) * C::kSfBytes, C::kSfBytes, bf);
+                bulk_load(st + C::sKsf, p.k_sf + static_cast<size_t>(bh * nkvt + j) * C::kSfBytes, C::kSfBytes, bf);
                 tma_load_2d(st + C::sV, &tm_v, j * 64, bh * D, bf);
                 bulk_load(st + C::sVsf, p.vt_sf + (static_cast<size_t>(bh) * (p.Np / 64) + 2 * j) * 512, C::kVsfBytes,
                           bf);
@@ -336,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (valid1)
                         tc_cp_32x128b_warpx4(tmem + C::tSfq1 + 4 * a, sdesc_sf_atom(base_s + C::oQsf1 + 512 * a));
                 }
-                ok = mbar_wait(bars + kBarKvFull + 0, 0, abort_flag);
+                if (nmax > 0) ok = mbar_wait(bars + kBarKvFull + 0, 0, abort_flag);
             }
-            if (ok) {
+            if (ok && nmax > 0) {
                 tc_fence_after();
                 copy_ksf(0);
                 if (n0 > 0) ok = issue_qk(0, 0);
@@ -415,11 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             const int col0 = j * kBlk + 64 * h;
             const bool tail = col0 + 64 > p.N;
-            const bool diag = p.causal && (col0 + 63 > tile * kBlk);
+            const bool diag = p.causal && (col0 + 63 > tile * kBlk + off);
             if (tail || diag) {
                 // columns col0 + k with k >= lim are masked for this row
                 int lim = p.N - col0;
-                if (p.causal) lim = min(lim, grow - col0 + 1);
+                if (p.causal) lim = min(lim, grow + off - col0 + 1);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
 #pragma unroll
@@ -447,7 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const float rmax = fmaxf(xs[r], xs[kBlk + r]);
-            const float m_new = fmaxf(m, __fmul_rn(rmax, c2));
+            // clamped below at -FLT_MAX: a row that has seen no key yet gets
+            // P = 0 and alpha = 0 (its O and l are still 0), never inf - inf
+            const float m_new = fmaxf(fmaxf(m, __fmul_rn(rmax, c2)), -3.402823466e38f);
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
             // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
@@ -548,15 +559,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
             tc_fence_after();
-            const float inv = __frcp_rn(l_row);
-            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.N + grow) * D + h * (D / 2);
+            const float inv = l_row > 0.0f ? __frcp_rn(l_row) : 0.0f;  // a row that sees no key outputs 0
+            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2);
 #pragma unroll
             for (int q = 0; q < D / 64; ++q) {
                 uint32_t o[32];
                 tmem_ld32(trow + tO + 32 * q, o);
                 tmem_ld_wait();
                 reg_fence32(o);
-                if (grow < p.N) {
+                if (grow < p.Nq) {
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -569,6 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
                 }
             }
+        } else if (ok && n_i == 0 && i <= static_cast<int>(valid1) && grow < p.Nq) {
+            // causal with more queries than keys: no row of this tile sees a key
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2));
+#pragma unroll
+            for (int v = 0; v < D / 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
     tc_fence_before();
@@ -589,7 +605,7 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     // Split the pairs of a last wave that would fill at most half of the SMs
     // into single-tile units (one CTA per SM).
     AttnParams q = p;
-    const int nqt = p.Np / kBlk;
+    const int nqt = p.Npq / kBlk;
     q.npairs = (nqt + 1) / 2;
     const int total = q.npairs * p.BH;
     int dev = 0, nsm = 148;

@@ -265,7 +265,8 @@ __device__ __forceinline__ void ksum_flush(double (&acc)[8], double *red, double
 
 // ------------------------------------------------------------- schedule
 // Work of the first launch for CTA g of G: a contiguous range of the Q and
-// V tiles (Q tiles of every (b, h) first, then V), then the K chunks
+// V tiles (Q tiles of every (b, h) first, then V; Q and V may have different
+// token counts), then the K chunks
 // g, g+G, g+2G, ... one tile at a time.  The Q/V ranges are sized so that
 // every CTA ends up with about the same number of tiles: CTAs holding one
 // K chunk more (the first nK % G) take tpc fewer Q/V tiles.
@@ -278,19 +279,20 @@ struct TileJob {
 };
 
 struct SchedA {
-    int ntile, nchunk, tpc, nqk;  // nqk = BH * ntile (Q tiles; V tiles follow)
+    int ntile_q, ntile, nchunk, tpc, nqk;  // nqk = BH * ntile_q (Q tiles; V tiles follow)
     int j, je;                    // Q/V tiles [j, je)
     int ki, nK, G;                // next K chunk item, items, stride
     int kbh, kch, kt, kt_end;     // current K chunk and its tiles [kt, kt_end)
 
-    __host__ __device__ void init(int BH, int ntile_, int nchunk_, int tpc_, int g, int G_) {
+    __host__ __device__ void init(int BH, int ntile_q_, int ntile_, int nchunk_, int tpc_, int g, int G_) {
+        ntile_q = ntile_q_;
         ntile = ntile_;
         nchunk = nchunk_;
         tpc = tpc_;
-        nqk = BH * ntile;
+        nqk = BH * ntile_q;
         G = G_;
         nK = BH * nchunk;
-        const int nqv = 2 * nqk;
+        const int nqv = nqk + BH * ntile;
         const int a = nK / G, r = nK % G;
         (void)a;
         long long q_hi = (static_cast<long long>(nqv) + static_cast<long long>(r) * tpc + G - 1) / G;
@@ -311,9 +313,10 @@ struct SchedA {
         if (j < je) {
             const int kind = j < nqk ? 0 : 1;
             const int jj = kind ? j - nqk : j;
+            const int nt = kind ? ntile : ntile_q;
             t.kind = kind;
-            t.bh = jj / ntile;
-            t.tile = jj % ntile;
+            t.bh = jj / nt;
+            t.tile = jj % nt;
             t.chunk = 0;
             t.last = false;
             ++j;
@@ -401,9 +404,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     extern __shared__ uint8_t smem_raw[];
     pdl_trigger();  // the second launch may start once every CTA of this one has
     const SmemPtrs sm = smem_setup<D>(smem_raw);
-    const int ntile = p.Np / kTile;
     SchedA prod, cons;
-    prod.init(p.BH, ntile, p.nchunk, p.chunk / kTile, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
+    prod.init(p.BH, p.Npq / kTile, p.Np / kTile, p.nchunk, p.chunk / kTile, static_cast<int>(blockIdx.x),
+              static_cast<int>(gridDim.x));
     cons = prod;
     const uint64_t pol_once = l2_policy_evict_first();
     const uint64_t pol_k = l2_policy_evict_normal();
@@ -432,8 +435,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         const uint8_t *st = sm.base + s * QCfg<D>::kTileBytes;
         if (t.kind == 0) {
-            qk_tile<D, false>(st, p.N, t.tile, nullptr, sm.lut, p.q_fp4 + static_cast<size_t>(t.bh) * p.Np * (D / 2),
-                              p.q_sf + static_cast<size_t>(t.bh) * p.Np * (D / 16));
+            qk_tile<D, false>(st, p.Nq, t.tile, nullptr, sm.lut,
+                              p.q_fp4 + static_cast<size_t>(t.bh) * p.Npq * (D / 2),
+                              p.q_sf + static_cast<size_t>(t.bh) * p.Npq * (D / 16));
         } else if (t.kind == 1) {
             v_tile<D>(st, p.Np, t.tile, sm.lut, p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
                       p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
@@ -532,7 +536,8 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const long long ntile = p.Np / kTile;
-    const long long work_a = 2 * p.BH * ntile + static_cast<long long>(p.BH) * p.nchunk;
+    const long long work_a = static_cast<long long>(p.BH) * (p.Npq / kTile + ntile) +
+                             static_cast<long long>(p.BH) * p.nchunk;
     const long long slots = static_cast<long long>(nsm) * kCtasPerSm;
     const int grid_a = static_cast<int>(work_a < slots ? work_a : slots);
     quant_qvk_kernel<D><<<grid_a, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
@@ -555,8 +560,8 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
 }  // namespace quant
 
 // Two launches: Q/V tiles and K chunk sums, then smoothed K tiles.  tq, tk,
-// tv: 3-D bf16 tensor maps {d, N, B*H} with 64 x 128 boxes and 128-byte
-// swizzle.
+// tv: 3-D bf16 tensor maps {d, tokens, B*H} (Nq tokens for Q, N for K and V)
+// with 64 x 128 boxes and 128-byte swizzle.
 inline cudaError_t launch_quant(const QuantParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, int d, cudaStream_t stream) {
     return d == 128 ? quant::launch_d<128>(p, tq, tk, tv, stream) : quant::launch_d<64>(p, tq, tk, tv, stream);

@@ -131,13 +131,14 @@ extern "C" {
 
 const char *sa3_version(void) { return "libsa3 0.1.0 (sm_100a)"; }
 
-int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, int N, int d,
-                     const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes, struct CUstream_st *stream) {
-    int rc = check_shape(B, H, N, d);
-    if (rc != SA3_OK) return rc;
+int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, int H, int Nq, int Nkv, int d,
+                          const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes,
+                          struct CUstream_st *stream) {
+    int rc = check_shape(B, H, Nq, d);
+    if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
     if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
     if ((rc = check_qkv(out)) != SA3_OK) return rc;
-    const int64_t need = sa3_quant_workspace_bytes(B, H, N, d);
+    const int64_t need = sa3_quant_workspace_bytes(B, H, Nkv, d);
     if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
     sa3::QuantParams p;
     p.q_fp4 = static_cast<uint8_t *>(out->q_fp4);
@@ -149,15 +150,23 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, 
     p.k_mean = out->k_mean;
     p.part = static_cast<double *>(workspace);
     p.BH = B * H;
-    p.N = N;
-    p.Np = static_cast<int>(sa3_padded_len(N));
-    p.chunk = static_cast<int>(sa3_kmean_chunk(N));
-    p.nchunk = static_cast<int>(sa3_kmean_nchunk(N));
+    p.N = Nkv;
+    p.Np = static_cast<int>(sa3_padded_len(Nkv));
+    p.Nq = Nq;
+    p.Npq = static_cast<int>(sa3_padded_len(Nq));
+    p.chunk = static_cast<int>(sa3_kmean_chunk(Nkv));
+    p.nchunk = static_cast<int>(sa3_kmean_nchunk(Nkv));
     CUtensorMap tq, tk, tv;
-    if (!make_qkv_map(&tq, q, d, N, p.BH) || !make_qkv_map(&tk, k, d, N, p.BH) || !make_qkv_map(&tv, v, d, N, p.BH))
+    if (!make_qkv_map(&tq, q, d, Nq, p.BH) || !make_qkv_map(&tk, k, d, Nkv, p.BH) ||
+        !make_qkv_map(&tv, v, d, Nkv, p.BH))
         return SA3_ERR_CUDA;
     return sa3::launch_quant(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK
                                                                                                         : SA3_ERR_CUDA;
+}
+
+int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, int N, int d,
+                     const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes, struct CUstream_st *stream) {
+    return sa3_quantize_qkv_lens(q, k, v, B, H, N, N, d, out, workspace, workspace_bytes, stream);
 }
 
 int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B, int H, int N, int d,
@@ -175,19 +184,20 @@ int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B,
     return sa3_quantize_qkv(q, k, v, B, H, N, d, out, scratch, SA3_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,
-                 struct CUstream_st *stream) {
-    int rc = check_shape(B, H, N, d);
-    if (rc != SA3_OK) return rc;
+int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                      void *out, struct CUstream_st *stream) {
+    int rc = check_shape(B, H, Nq, d);
+    if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
     if ((rc = check_qkv(in)) != SA3_OK) return rc;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
     const int BH = B * H;
-    const int Np = static_cast<int>(sa3_padded_len(N));
+    const int Npq = static_cast<int>(sa3_padded_len(Nq));
+    const int Np = static_cast<int>(sa3_padded_len(Nkv));
     CUtensorMap tq, tk, tv;
     const CUtensorMapSwizzle qk_sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-    if (!make_map(&tq, in->q_fp4, d / 2, static_cast<uint64_t>(BH) * Np, d / 2, 128, qk_sw) ||
+    if (!make_map(&tq, in->q_fp4, d / 2, static_cast<uint64_t>(BH) * Npq, d / 2, 128, qk_sw) ||
         !make_map(&tk, in->k_fp4, d / 2, static_cast<uint64_t>(BH) * Np, d / 2, 128, qk_sw) ||
         !make_map(&tv, in->vt_fp4, Np / 2, static_cast<uint64_t>(BH) * d, 64, d, CU_TENSOR_MAP_SWIZZLE_64B))
         return SA3_ERR_CUDA;
@@ -197,13 +207,20 @@ int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, 
     p.vt_sf = static_cast<const uint8_t *>(in->vt_sf);
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.BH = BH;
-    p.N = N;
+    p.N = Nkv;
     p.Np = Np;
+    p.Nq = Nq;
+    p.Npq = Npq;
     p.causal = causal;
     p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
     return sa3::launch_attn(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA3_OK
                : SA3_ERR_CUDA;
+}
+
+int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,
+                 struct CUstream_st *stream) {
+    return sa3_attn_fwd_lens(in, B, H, N, N, d, causal, sm_scale, out, stream);
 }
 
 int sa3_selftest_wait_timeout(unsigned int limit_us, struct CUstream_st *stream) {

@@ -20,8 +20,10 @@ struct QuantParams {
     float *k_mean;
     double *part;  // [BH][nchunk][d] scratch: fp64 column sums of K per chunk
     int BH;
-    int N;
-    int Np;
+    int N;       // K and V tokens
+    int Np;      // N rounded up to 128
+    int Nq;      // Q tokens (== N for self-attention)
+    int Npq;     // Nq rounded up to 128
     int nchunk;  // fp64 partial sums of K per (b, h)
     int chunk;   // tokens per partial sum
 };
@@ -32,9 +34,11 @@ struct AttnParams {
     const uint8_t *vt_sf;
     __nv_bfloat16 *out;
     int BH;
-    int N;
-    int Np;
-    int causal;
+    int N;             // key / value tokens
+    int Np;            // N rounded up to 128
+    int Nq;            // query tokens (== N for self-attention)
+    int Npq;           // Nq rounded up to 128
+    int causal;        // mask col > row + N - Nq
     float scale_log2;  // fp32(sm_scale * log2 e)
     int npairs;        // Q-tile pairs per head (set by the launcher)
     int pair_units;    // work units that are pairs; the rest are single tiles

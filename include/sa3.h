@@ -155,6 +155,36 @@ int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d,
                  struct CUstream_st *stream);
 
 /*
+ * sa3_quantize_qkv_lens, sa3_attn_fwd_lens -- the two calls above with a
+ * query length Nq that may differ from the key/value length Nkv (cross
+ * attention, decoding against a longer key/value sequence, chunked prefill).
+ * The pages define the method for one sequence; these take its plainest
+ * extension, used by the FlashAttention family in the same reference list:
+ *
+ *   q          : bf16 [B][H][Nq][d];  k, v : bf16 [B][H][Nkv][d].
+ *   out / in   : q_fp4, q_sf sized with Nq (sa3_qk_fp4_bytes(B, H, Nq, d),
+ *                sa3_qk_sf_bytes(B, H, Nq, d)); k_fp4, k_sf, vt_fp4, vt_sf
+ *                sized with Nkv; the K mean runs over the Nkv keys;
+ *                workspace: sa3_quant_workspace_bytes(B, H, Nkv, d).
+ *   causal = 1 : query row r sees keys 0 .. r + Nkv - Nq (the last query is
+ *                aligned with the last key; for Nq == Nkv the usual mask).
+ *                A row that sees no key (r + Nkv - Nq < 0) outputs 0.
+ *   out (attn) : bf16 [B][H][Nq][d].
+ *
+ * Everything else -- block recipe, arguments, errors, asynchrony -- is as in
+ * sa3_quantize_qkv / sa3_attn_fwd, which are these calls with Nq == Nkv.
+ * Both lengths obey the shape limits at the top of this file.
+ */
+int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v,
+                          int B, int H, int Nq, int Nkv, int d,
+                          const sa3_qkv_fp4 *out,
+                          void *workspace, size_t workspace_bytes,
+                          struct CUstream_st *stream);
+int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d,
+                      int causal, float sm_scale, void *out,
+                      struct CUstream_st *stream);
+
+/*
  * sa3_quantize_qkv_noalloc -- sa3_quantize_qkv without a caller workspace.
  *
  * There is no counterpart in the paper: this is a convenience for callers

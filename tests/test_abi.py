@@ -26,8 +26,9 @@ def lib():
 
 
 def test_header_declares_the_boundary():
-    assert _declared() == ["sa3_attn_fwd", "sa3_device_status", "sa3_quantize_qkv",
-                           "sa3_quantize_qkv_noalloc", "sa3_selftest_wait_timeout", "sa3_version"]
+    assert _declared() == ["sa3_attn_fwd", "sa3_attn_fwd_lens", "sa3_device_status", "sa3_quantize_qkv",
+                           "sa3_quantize_qkv_lens", "sa3_quantize_qkv_noalloc", "sa3_selftest_wait_timeout",
+                           "sa3_version"]
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -58,3 +59,13 @@ def test_argument_checks_need_no_gpu(lib):
     lib.sa3_selftest_wait_timeout.restype = I
     lib.sa3_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     assert lib.sa3_selftest_wait_timeout(0, None) == 1
+    # separate query / key lengths: each is checked
+    lib.sa3_quantize_qkv_lens.restype = I
+    lib.sa3_quantize_qkv_lens.argtypes = [P, P, P, I, I, I, I, I, P, P, ctypes.c_size_t, P]
+    lib.sa3_attn_fwd_lens.restype = I
+    lib.sa3_attn_fwd_lens.argtypes = [P, I, I, I, I, I, I, ctypes.c_float, P, P]
+    assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 8, 0, 64, None, None, 0, None) == 1
+    assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 0, 8, 64, None, None, 0, None) == 1
+    assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 8, 8, 96, None, None, 0, None) == 2
+    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 0, 64, 0, 0.0, None, None) == 1
+    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 8, 64, 0, 0.0, None, None) == 1
