@@ -147,7 +147,10 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
-template <int D>
+// kCross: query and key/value lengths differ (bottom-right causal offset,
+// rows that may see no key); false compiles the self-attention case with
+// those terms folded away.
+template <int D, bool kCross>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // what would otherwise be a short last wave.
     const int nqt = p.Npq / kBlk;   // Q tiles
     const int nkvt = p.Np / kBlk;   // KV blocks
-    const int off = p.N - p.Nq;     // causal: row r sees keys 0 .. r + off
+    const int off = kCross ? p.N - p.Nq : 0;  // causal: row r sees keys 0 .. r + off
     const int u = static_cast<int>(blockIdx.x);
     const bool single = u >= p.pair_units;
     const int pu = single ? p.pair_units + (u - p.pair_units) / 2 : u;
@@ -456,9 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const float rmax = fmaxf(xs[r], xs[kBlk + r]);
-            // clamped below at -FLT_MAX: a row that has seen no key yet gets
-            // P = 0 and alpha = 0 (its O and l are still 0), never inf - inf
-            const float m_new = fmaxf(fmaxf(m, __fmul_rn(rmax, c2)), -3.402823466e38f);
+            // (kCross) clamped below at -FLT_MAX: a row that has seen no key yet
+            // gets P = 0 and alpha = 0 (its O and l are still 0), never inf - inf
+            const float m_new = kCross ? fmaxf(fmaxf(m, __fmul_rn(rmax, c2)), -3.402823466e38f)
+                                       : fmaxf(m, __fmul_rn(rmax, c2));
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
             // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
@@ -559,7 +563,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
             tc_fence_after();
-            const float inv = l_row > 0.0f ? __frcp_rn(l_row) : 0.0f;  // a row that sees no key outputs 0
+            // a row that sees no key (kCross only) outputs 0
+            const float inv = (!kCross || l_row > 0.0f) ? __frcp_rn(l_row) : 0.0f;
             __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2);
 #pragma unroll
             for (int q = 0; q < D / 64; ++q) {
@@ -580,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
                 }
             }
-        } else if (ok && n_i == 0 && i <= static_cast<int>(valid1) && grow < p.Nq) {
+        } else if (kCross && ok && n_i == 0 && i <= static_cast<int>(valid1) && grow < p.Nq) {
             // causal with more queries than keys: no row of this tile sees a key
             uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2));
 #pragma unroll
@@ -599,8 +604,9 @@ template <int D>
 cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      cudaStream_t stream) {
     using C = Cfg<D>;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+    const bool cross = p.Nq != p.N;
+    auto kernel = cross ? attn_fwd_kernel<D, true> : attn_fwd_kernel<D, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // Split the pairs of a last wave that would fill at most half of the SMs
     // into single-tile units (one CTA per SM).
@@ -614,7 +620,7 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;
     const dim3 grid(q.pair_units + 2 * split);
-    attn_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
+    kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
     return cudaGetLastError();
 }
 
