@@ -72,9 +72,9 @@ def _load():
         lib.oracle_kmean.restype = None
         lib.oracle_kmean.argtypes = [P, I, I, I, I, P]
         lib.oracle_quantize_qkv.restype = None
-        lib.oracle_quantize_qkv.argtypes = [P, P, P, I, I, I, I, I, I] + [P] * 7
+        lib.oracle_quantize_qkv.argtypes = [P, P, P, I, I, I, I, I, I, I] + [P] * 8
         lib.oracle_attn_fwd.restype = None
-        lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, I, F, P, I, P]
+        lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, I, F, I, P, P, I, P]
         lib.oracle_attn_exact.restype = None
         lib.oracle_attn_exact.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, I, P]
         lib.oracle_num_threads.restype = I
@@ -136,11 +136,12 @@ def kmean(k) -> np.ndarray:
     return out
 
 
-def quantize_qkv(q, k, v, smooth_k: bool = True) -> dict:
+def quantize_qkv(q, k, v, smooth_k: bool = True, smooth_v: bool = False) -> dict:
     """Returns canonical-layout arrays: q_codes [B,H,Np(Nq),d/2], q_sf
     [B,H,Np(Nq),d/16], k_codes/k_sf the same over Np(Nkv), vt_codes
     [B,H,d,Np(Nkv)/2], vt_sf [B,H,d,Np(Nkv)/16], k_mean [B,H,d]; and the
-    lengths n_q, n_kv.  q is [B,H,Nq,d], k and v are [B,H,Nkv,d]."""
+    lengths n_q, n_kv; with smooth_v also v_mean [B,H,d] (V quantized after
+    subtracting it).  q is [B,H,Nq,d], k and v are [B,H,Nkv,d]."""
     q, k, v = _as_u16(q), _as_u16(k), _as_u16(v)
     B, H, Nq, d = q.shape
     N = k.shape[2]
@@ -155,11 +156,14 @@ def quantize_qkv(q, k, v, smooth_k: bool = True) -> dict:
         vt_codes=np.zeros((B, H, d, Np // 2), np.uint8),
         vt_sf=np.zeros((B, H, d, Np // VEC), np.uint8),
         k_mean=np.zeros((B, H, d), np.float32),
+        v_mean=np.zeros((B, H, d), np.float32),
     )
     _load().oracle_quantize_qkv(
-        _ptr(q), _ptr(k), _ptr(v), B, H, Nq, N, d, int(bool(smooth_k)),
+        _ptr(q), _ptr(k), _ptr(v), B, H, Nq, N, d, int(bool(smooth_k)), int(bool(smooth_v)),
         _ptr(r["q_codes"]), _ptr(r["q_sf"]), _ptr(r["k_codes"]), _ptr(r["k_sf"]),
-        _ptr(r["vt_codes"]), _ptr(r["vt_sf"]), _ptr(r["k_mean"]))
+        _ptr(r["vt_codes"]), _ptr(r["vt_sf"]), _ptr(r["k_mean"]), _ptr(r["v_mean"]))
+    if not smooth_v:
+        del r["v_mean"]
     r["n_q"], r["n_kv"] = Nq, N
     return r
 
@@ -172,12 +176,14 @@ def _units_arr(units):
 
 
 def attn_fwd(qz: dict, N: int, causal: bool, sm_scale: float | None = None,
-             units=None, out: np.ndarray | None = None, n_kv: int | None = None) -> np.ndarray:
+             units=None, out: np.ndarray | None = None, n_kv: int | None = None,
+             p_two_level: bool = False) -> np.ndarray:
     """Tiled FP4 attention on canonical-layout quantized operands with N
     query rows and ``n_kv`` key columns (default: qz["n_kv"] if present,
     else N).  Returns bf16 bits uint16 [B,H,N,d]; rows outside ``units``
     stay as in ``out`` (zeros by default).  ``units`` lists (b*H+h,
-    q_block) pairs."""
+    q_block) pairs.  p_two_level: P pre-scaled by 2^11 before microscaling
+    (R14); qz["v_mean"], if present, is added back after O / l (R13)."""
     if n_kv is None:
         n_kv = qz.get("n_kv", N)
     B, H, Np, dh = qz["q_codes"].shape
@@ -189,8 +195,11 @@ def attn_fwd(qz: dict, N: int, causal: bool, sm_scale: float | None = None,
     u, nu = _units_arr(units)
     arrs = [np.ascontiguousarray(qz[n]) for n in
             ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf")]
+    vm = qz.get("v_mean")
+    if vm is not None:
+        vm = np.ascontiguousarray(vm, dtype=np.float32)
     _load().oracle_attn_fwd(*[_ptr(a) for a in arrs], B, H, N, n_kv, d, int(bool(causal)),
-                            float(sm_scale), _ptr(u), nu, _ptr(out))
+                            float(sm_scale), int(bool(p_two_level)), _ptr(vm), _ptr(u), nu, _ptr(out))
     return out
 
 

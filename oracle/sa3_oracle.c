@@ -47,7 +47,13 @@
  *  R11 Q may have fewer or more tokens (Nq) than K and V (Nkv); the causal
  *     mask then aligns the last query with the last key (for Nq == Nkv this
  *     is the usual lower-triangular mask);
- *  R12 a query row that sees no key at all (causal, Nq > Nkv) outputs 0.
+ *  R12 a query row that sees no key at all (causal, Nq > Nkv) outputs 0;
+ *  R13 (optional) V smoothing: V_s = fp32(V) - mean of V over the keys,
+ *     quantized like V; out = bf16(O / l + mean) in fp32;
+ *  R14 (optional) two-level P: P' = P * 2^11 (the largest power of two with
+ *     2^k / 6 <= 448, so no block scale saturates) is microscaled instead of
+ *     P, and out = bf16((O / l) * 2^-11); being exact in binary, the
+ *     pre-scale changes only blocks whose E4M3 scale was subnormal or 0.
  */
 #include <math.h>
 #include <stdint.h>
@@ -212,8 +218,11 @@ void oracle_kmean(const uint16_t *k, int B, int H, int N, int d, float *mean)
  *   vt_codes         : [B*H][d][Np(Nkv)/2]   bytes (V transposed)
  *   vt_sf            : [B*H][d][Np(Nkv)/16]  E4M3 bytes
  *   k_mean           : [B*H][d] fp32, the mean over the Nkv tokens of K
+ *   v_mean           : [B*H][d] fp32, the same for V (smooth_v only)
  * Padding tokens get code 0 and scale byte 0.
- * smooth_k = 0 skips the subtraction (used to measure what smoothing buys). */
+ * smooth_k = 0 skips the subtraction (used to measure what smoothing buys).
+ * smooth_v = 1 quantizes V_s = fp32(V) - mean of V over the Nkv tokens, the
+ * same recipe as K (R13); attention adds the mean back after O / l. */
 static void quant_rows(const uint16_t *x_in, long bh, int N, int Np, int d, const float *sub,
                        uint8_t *codes_out, uint8_t *sf_out)
 {
@@ -234,16 +243,17 @@ static void quant_rows(const uint16_t *x_in, long bh, int N, int Np, int d, cons
 }
 
 void oracle_quantize_qkv(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                         int B, int H, int Nq, int Nkv, int d, int smooth_k,
+                         int B, int H, int Nq, int Nkv, int d, int smooth_k, int smooth_v,
                          uint8_t *q_codes, uint8_t *q_sf,
                          uint8_t *k_codes, uint8_t *k_sf,
-                         uint8_t *vt_codes, uint8_t *vt_sf, float *k_mean)
+                         uint8_t *vt_codes, uint8_t *vt_sf, float *k_mean, float *v_mean)
 {
     tables_init();
     const long BH = (long)B * H;
     const int Npq = oracle_padded_len(Nq);
     const int Np = oracle_padded_len(Nkv);
     oracle_kmean(k, B, H, Nkv, d, k_mean);
+    if (smooth_v) oracle_kmean(v, B, H, Nkv, d, v_mean);
 
     memset(q_codes, 0, (size_t)BH * Npq * d / 2);
     memset(q_sf, 0, (size_t)BH * Npq * d / VEC);
@@ -264,7 +274,8 @@ void oracle_quantize_qkv(const uint16_t *q, const uint16_t *k, const uint16_t *v
             for (int tb = 0; tb < Np / VEC; ++tb) {
                 for (int i = 0; i < VEC; ++i) {
                     int t = tb * VEC + i;
-                    x[i] = (t < Nkv) ? bf16_to_f32(v[(bh * Nkv + t) * d + c]) : 0.0f;
+                    float vv = (t < Nkv) ? bf16_to_f32(v[(bh * Nkv + t) * d + c]) : 0.0f;
+                    x[i] = (t < Nkv && smooth_v) ? vv - v_mean[bh * d + c] : vv;
                 }
                 int sc = quant_block(x, codes);
                 vt_sf[(bh * d + c) * (Np / VEC) + tb] = (uint8_t)sc;
@@ -288,15 +299,19 @@ static double deq(const uint8_t *codes, const uint8_t *sf, long elem, long sf_id
  * Nq query rows, Nkv key/value columns.  causal masks col > row + Nkv - Nq
  * (the last query row aligned with the last key, R11); a row that sees no
  * column at all gets output 0 (R12).
+ * p_two_level: P is scaled by 2^11 before it is microscaled and the output
+ * by 2^-11 after O / l (R14); v_mean (NULL: none) is added after O / l (R13).
  * units: n_units pairs (bh, q_block); NULL means every (bh, q_block).
  * out: bf16 [B*H][Nq][d]; only rows of the listed units are written. */
 void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                      const uint8_t *k_codes, const uint8_t *k_sf,
                      const uint8_t *vt_codes, const uint8_t *vt_sf,
                      int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                     int p_two_level, const float *v_mean,
                      const int32_t *units, int n_units, uint16_t *out)
 {
     tables_init();
+    const float p_pre = p_two_level ? 2048.0f : 1.0f;   /* 2^11, exact (R14) */
     const long BH = (long)B * H;
     const int Npq = oracle_padded_len(Nq);
     const int Np = oracle_padded_len(Nkv);
@@ -368,9 +383,12 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                 for (int i = 0; i < BLK; ++i) psum += p[i];
                 rowsum = (float)psum;
                 l = alpha * l + rowsum;
-                /* Quantize P per 16-column block (R3, R8). */
+                /* Quantize P per 16-column block (R3, R8), after the exact
+                 * two-level pre-scale when asked for (R14). */
+                float pp[BLK];
+                for (int i = 0; i < BLK; ++i) pp[i] = p[i] * p_pre;
                 for (int b = 0; b < BLK / VEC; ++b) {
-                    int sc = quant_block(p + b * VEC, codes);
+                    int sc = quant_block(pp + b * VEC, codes);
                     for (int i = 0; i < VEC; ++i)
                         phat[b * VEC + i] = g_e2m1[codes[i]] * g_e4m3[sc];
                 }
@@ -383,8 +401,16 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                 }
                 m = m_new;
             }
-            for (int c = 0; c < d; ++c)
-                out[(bh * Nq + row) * d + c] = l > 0.0f ? oracle_f32_to_bf16(O[c] / l) : 0;
+            for (int c = 0; c < d; ++c) {
+                if (!(l > 0.0f)) {
+                    out[(bh * Nq + row) * d + c] = 0;
+                    continue;
+                }
+                float o = O[c] / l;
+                if (p_two_level) o = o * (1.0f / 2048.0f);  /* exact */
+                if (v_mean) o = o + v_mean[bh * d + c];
+                out[(bh * Nq + row) * d + c] = oracle_f32_to_bf16(o);
+            }
         }
         free(qrow);
         free(khat);
