@@ -26,6 +26,7 @@ SA3_ERR_INVALID_ARG = 1
 SA3_ERR_UNSUPPORTED = 2
 SA3_ERR_CUDA = 3
 SA3_ERR_TIMEOUT = 4
+SA3_P_TWO_LEVEL = 1
 _NAMES = {0: "SA3_OK", 1: "SA3_ERR_INVALID_ARG", 2: "SA3_ERR_UNSUPPORTED", 3: "SA3_ERR_CUDA",
           4: "SA3_ERR_TIMEOUT"}
 
@@ -68,7 +69,7 @@ def lib() -> ctypes.CDLL:
             L.sa3_quantize_qkv_lens.restype = I
             L.sa3_quantize_qkv_lens.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(_QKV), P, ctypes.c_size_t, P]
             L.sa3_attn_fwd_lens.restype = I
-            L.sa3_attn_fwd_lens.argtypes = [ctypes.POINTER(_QKV), I, I, I, I, I, I, F, P, P]
+            L.sa3_attn_fwd_lens.argtypes = [ctypes.POINTER(_QKV), I, I, I, I, I, I, F, ctypes.c_uint, P, P]
             L.sa3_device_status.restype = I
             L.sa3_device_status.argtypes = [P]
             _lib = L
@@ -178,22 +179,24 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 
 def attn_fwd(qz: QuantizedQKV, causal: bool = False, sm_scale: float | None = None,
-             out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+             out: torch.Tensor | None = None, stream=None, p_two_level: bool = False) -> torch.Tensor:
     """sa3_attn_fwd: FP4 attention of quantized operands; bf16 [B,H,Nq,d].
     With Nq != N (sa3_attn_fwd_lens) the causal mask aligns the last query
-    with the last key; a row that sees no key is 0."""
+    with the last key; a row that sees no key is 0.  p_two_level: P scaled
+    by 2^11 before it is microscaled (SA3_P_TWO_LEVEL)."""
     B, H, N, d, Nq = qz.B, qz.H, qz.N, qz.d, qz.n_q
     if out is None:
         out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=qz.q_fp4.device)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     st = qz.struct()
-    if Nq == N:
+    if Nq == N and not p_two_level:
         rc = lib().sa3_attn_fwd(ctypes.byref(st), B, H, N, d, int(bool(causal)), float(sm_scale),
                                 out.data_ptr(), _stream_ptr(stream))
     else:
+        flags = SA3_P_TWO_LEVEL if p_two_level else 0
         rc = lib().sa3_attn_fwd_lens(ctypes.byref(st), B, H, Nq, N, d, int(bool(causal)), float(sm_scale),
-                                     out.data_ptr(), _stream_ptr(stream))
+                                     flags, out.data_ptr(), _stream_ptr(stream))
     if rc != SA3_OK:
         raise Sa3Error(rc, "sa3_attn_fwd")
     return out

@@ -74,7 +74,7 @@ struct Cfg {
     static constexpr int oP1 = oP0 + kPBytes;
     static constexpr int oPsf0 = oP1 + kPBytes;
     static constexpr int oPsf1 = oPsf0 + kPsfBytes;
-    static constexpr int oLut = oPsf1 + kPsfBytes;     // 2 x 256 floats: log2(1/s), s per E4M3 code s
+    static constexpr int oLut = oPsf1 + kPsfBytes;     // 2 x 256 floats: log2(2^pre / s), s per E4M3 code s
     static constexpr int oXch = oLut + 2048;           // row maxima [2 parity][2 tiles][2 halves][128]
     static constexpr int oXl = oXch + 4096;            // row sums [2 tiles][2 halves][128]
     static constexpr int oBar = oXl + 2048;
@@ -148,9 +148,10 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // kCross: query and key/value lengths differ (bottom-right causal offset,
-// rows that may see no key); false compiles the self-attention case with
-// those terms folded away.
-template <int D, bool kCross>
+// rows that may see no key).  kTwo: P is pre-scaled by 2^11 before it is
+// microscaled (two-level P).  Each term is compiled only into the instances
+// that use it.
+template <int D, bool kCross, bool kTwo>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -216,9 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // which the saturating conversion never produces) map to log2 = 0,
         // s = 1: such a block holds only P < 6 * 2^-10, whose codes at scale
         // 1 are all 0, exactly as at scale 0, and whose row-sum terms stay P.
+        // kTwo: every log2 entry gains the pre-scale exponent 11, so that
+        // y = P * 2^11 / s (and y = P * 2^11 for code 0, whose P' is still
+        // below 6 * 2^-10 and quantizes to 0)
         const float v = e4m3_value(threadIdx.x);
         const bool unit = v == 0.0f || v != v;
-        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] = unit ? 0.0f : -log2f(v);
+        const float pre = kTwo ? 11.0f : 0.0f;
+        reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] = unit ? pre : pre - log2f(v);
         reinterpret_cast<float *>(base + C::oLut)[256 + threadIdx.x] = unit ? 1.0f : v;
     }
     if (warp == kWarpMma) {
@@ -463,6 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // gets P = 0 and alpha = 0 (its O and l are still 0), never inf - inf
             const float m_new = kCross ? fmaxf(fmaxf(m, __fmul_rn(rmax, c2)), -3.402823466e38f)
                                        : fmaxf(m, __fmul_rn(rmax, c2));
+            // -m' plus the optional two-level pre-scale exponent (0 or 11):
+            // P' = P * 2^pre is what gets microscaled; l and O both carry the
+            // 2^pre, so O / l needs no correction
             const float nm = -m_new;
             const float alpha = ex2(__fsub_rn(m, m_new));
             // block scales: s_b = E4M3(amax_b / 6) with amax_b = 2^(bm_b*c - m'),
@@ -471,9 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             float lg[4], sv[4];
 #pragma unroll
             for (int b = 0; b < 4; b += 2) {
-                const float a0 = ex2(__fsub_rn(__fmul_rn(bm[b], c2), m_new));
-                const float a1 = ex2(__fsub_rn(__fmul_rn(bm[b + 1], c2), m_new));
-                const uint32_t sc2 = cvt_e4m3x2(a1 * kSixth, a0 * kSixth);  // byte 0: block b
+                const float a0 = ex2(__fadd_rn(__fmul_rn(bm[b], c2), nm));
+                const float a1 = ex2(__fadd_rn(__fmul_rn(bm[b + 1], c2), nm));
+                // amax' / 6 with amax' = 2^11 * amax under kTwo (exact: 2^11 * fp32(1/6))
+                constexpr float kDiv = kTwo ? 2048.0f * kSixth : kSixth;
+                const uint32_t sc2 = cvt_e4m3x2(a1 * kDiv, a0 * kDiv);  // byte 0: block b
                 lg[b] = lg_lut[sc2 & 0xFF];
                 lg[b + 1] = lg_lut[sc2 >> 8];
                 sv[b] = sv_lut[sc2 & 0xFF];
@@ -605,7 +615,9 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
                      cudaStream_t stream) {
     using C = Cfg<D>;
     const bool cross = p.Nq != p.N;
-    auto kernel = cross ? attn_fwd_kernel<D, true> : attn_fwd_kernel<D, false>;
+    const bool two = p.p_pre_log2 != 0.0f;
+    auto kernel = cross ? (two ? attn_fwd_kernel<D, true, true> : attn_fwd_kernel<D, true, false>)
+                        : (two ? attn_fwd_kernel<D, false, true> : attn_fwd_kernel<D, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // Split the pairs of a last wave that would fill at most half of the SMs

@@ -185,11 +185,12 @@ int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B,
 }
 
 int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
-                      void *out, struct CUstream_st *stream) {
+                      unsigned int flags, void *out, struct CUstream_st *stream) {
     int rc = check_shape(B, H, Nq, d);
     if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
     if ((rc = check_qkv(in)) != SA3_OK) return rc;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL)) != 0) return SA3_ERR_INVALID_ARG;
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
     const int BH = B * H;
@@ -213,6 +214,7 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
     p.Npq = Npq;
     p.causal = causal;
     p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+    p.p_pre_log2 = (flags & SA3_P_TWO_LEVEL) ? 11.0f : 0.0f;
     return sa3::launch_attn(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA3_OK
                : SA3_ERR_CUDA;
@@ -220,7 +222,7 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
 
 int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,
                  struct CUstream_st *stream) {
-    return sa3_attn_fwd_lens(in, B, H, N, N, d, causal, sm_scale, out, stream);
+    return sa3_attn_fwd_lens(in, B, H, N, N, d, causal, sm_scale, 0u, out, stream);
 }
 
 int sa3_selftest_wait_timeout(unsigned int limit_us, struct CUstream_st *stream) {

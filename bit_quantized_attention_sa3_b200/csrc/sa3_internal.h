@@ -40,6 +40,8 @@ struct AttnParams {
     int Npq;           // Nq rounded up to 128
     int causal;        // mask col > row + N - Nq
     float scale_log2;  // fp32(sm_scale * log2 e)
+    float p_pre_log2;  // 0, or 11 for two-level P (P scaled by 2^11 before microscaling;
+                       // selects the kernel instance, whose exponent is fixed)
     int npairs;        // Q-tile pairs per head (set by the launcher)
     int pair_units;    // work units that are pairs; the rest are single tiles
 };

@@ -171,17 +171,27 @@ int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d,
  *                A row that sees no key (r + Nkv - Nq < 0) outputs 0.
  *   out (attn) : bf16 [B][H][Nq][d].
  *
+ * flags (attention): 0, or SA3_P_TWO_LEVEL -- P is scaled by 2^11 before it
+ *   is microscaled (the largest power of two with 2^k / 6 <= 448, so no
+ *   block scale saturates) and O / l is unchanged by it because l carries
+ *   the same factor.  Being exact in binary, the pre-scale changes only the
+ *   16-column blocks whose E4M3 scale would be subnormal or 0 (P below
+ *   6 * 2^-6 relative to the row maximum), which then keep 3 significant
+ *   scale bits.  The pages do not describe it: an accuracy option, off by
+ *   default.  Other bits: SA3_ERR_INVALID_ARG.
+ *
  * Everything else -- block recipe, arguments, errors, asynchrony -- is as in
- * sa3_quantize_qkv / sa3_attn_fwd, which are these calls with Nq == Nkv.
- * Both lengths obey the shape limits at the top of this file.
+ * sa3_quantize_qkv / sa3_attn_fwd, which are these calls with Nq == Nkv and
+ * flags 0.  Both lengths obey the shape limits at the top of this file.
  */
+#define SA3_P_TWO_LEVEL 1u
 int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v,
                           int B, int H, int Nq, int Nkv, int d,
                           const sa3_qkv_fp4 *out,
                           void *workspace, size_t workspace_bytes,
                           struct CUstream_st *stream);
 int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d,
-                      int causal, float sm_scale, void *out,
+                      int causal, float sm_scale, unsigned int flags, void *out,
                       struct CUstream_st *stream);
 
 /*

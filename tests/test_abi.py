@@ -63,9 +63,9 @@ def test_argument_checks_need_no_gpu(lib):
     lib.sa3_quantize_qkv_lens.restype = I
     lib.sa3_quantize_qkv_lens.argtypes = [P, P, P, I, I, I, I, I, P, P, ctypes.c_size_t, P]
     lib.sa3_attn_fwd_lens.restype = I
-    lib.sa3_attn_fwd_lens.argtypes = [P, I, I, I, I, I, I, ctypes.c_float, P, P]
+    lib.sa3_attn_fwd_lens.argtypes = [P, I, I, I, I, I, I, ctypes.c_float, ctypes.c_uint, P, P]
     assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 8, 0, 64, None, None, 0, None) == 1
     assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 0, 8, 64, None, None, 0, None) == 1
     assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 8, 8, 96, None, None, 0, None) == 2
-    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 0, 64, 0, 0.0, None, None) == 1
-    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 8, 64, 0, 0.0, None, None) == 1
+    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 0, 64, 0, 0.0, 0, None, None) == 1
+    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 8, 64, 0, 0.0, 0, None, None) == 1

@@ -1,0 +1,70 @@
+"""SA3_P_TWO_LEVEL on the GPU against the oracle with p_two_level=True.
+
+Bar as for the default recipe: output rel-L2 <= 2e-3 against the oracle on
+the same quantized operands, cosine against fp64 exact attention within
+1e-3 of the oracle's.  Covers the self-attention and the unequal-length
+kernel instances."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sa3_inputs
+from sa3_testutil import bits_to_f32, cosine, qk_sf_to_canonical, rel_l2, vt_sf_to_canonical
+
+sa3 = pytest.importorskip("bit_quantized_attention_sa3_b200")
+
+TOL = 2e-3
+
+CASES = [
+    ("tiny_b1h2n256d64", 300, 300, {"H": 3}),
+    ("noncausal_b2h16n4096d128", 640, 640, {"B": 2, "H": 2}),
+    ("videodit_b1h30n17776d64", 1000, 1000, {"H": 2}),
+    ("longctx_b1h32n32768d128_causal", 1024, 1024, {"H": 2}),
+    ("noncausal_b2h16n4096d128", 77, 1000, {"B": 1, "H": 2}),
+]
+
+
+def _ids(c):
+    return f"{c[0]}-q{c[1]}-kv{c[2]}"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["noncausal", "causal"])
+@pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
+def test_two_level_matches_oracle(case, causal):
+    name, Nq, Nkv, over = case
+    o = dict(over)
+    o["N"] = max(Nq, Nkv)
+    q, k, v = sa3_inputs.make_qkv(name, shape_override=o)
+    q, k, v = q[:, :, :Nq].contiguous(), k[:, :, :Nkv].contiguous(), v[:, :, :Nkv].contiguous()
+    B, H, _, d = q.shape
+    qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
+    out = sa3.attn_fwd(qz, causal=causal, p_two_level=True)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    Npq, Np = sa3.padded_len(Nq), sa3.padded_len(Nkv)
+    canon = dict(q_codes=qz.q_fp4.cpu().numpy(), k_codes=qz.k_fp4.cpu().numpy(), vt_codes=qz.vt_fp4.cpu().numpy(),
+                 q_sf=qk_sf_to_canonical(qz.q_sf.cpu().numpy(), B, H, Npq, d),
+                 k_sf=qk_sf_to_canonical(qz.k_sf.cpu().numpy(), B, H, Np, d),
+                 vt_sf=vt_sf_to_canonical(qz.vt_sf.cpu().numpy(), B, H, Np, d))
+    ref = bits_to_f32(oracle.attn_fwd(canon, Nq, causal, n_kv=Nkv, p_two_level=True))
+    ex = oracle.attn_exact(q, k, v, causal)
+    live = (np.arange(Nq) + (Nkv - Nq) >= 0) if causal else np.ones(Nq, bool)
+    g, r, e = got[:, :, live], ref[:, :, live], ex[:, :, live]
+    err = rel_l2(g, r)
+    assert err <= TOL, f"rel-L2 vs oracle {err:.3e}"
+    assert cosine(g, e) >= cosine(r, e) - 1e-3
+
+
+@pytest.mark.gpu
+def test_unknown_flag_bits_are_rejected():
+    q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64")]
+    qz = sa3.quantize_qkv(q, k, v)
+    out = torch.empty_like(q)
+    import ctypes
+    rc = sa3.lib().sa3_attn_fwd_lens(ctypes.byref(qz.struct()), 1, 2, 256, 256, 64, 0, 0.0, 2, out.data_ptr(),
+                                     torch.cuda.current_stream().cuda_stream)
+    assert rc == sa3.SA3_ERR_INVALID_ARG
