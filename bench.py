@@ -218,32 +218,55 @@ def run_sa3(args, rank, world, local):
     if sa3.device_status() != sa3.SA3_OK:
         raise RuntimeError("device wait gave up during the timed steps")
 
-    # end-to-end through the public API: pinned host in -> host out
+    # end-to-end through the public API: pinned host in -> host out, every
+    # step copying its inputs up and its output down.  Pipelined as a serving
+    # loop would run it: two buffer sets, uploads on one stream, kernels on
+    # the launching stream, downloads on a third, so that step i+1's upload
+    # and step i-1's download overlap step i's kernels.
     qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
-    out_h = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    sets = []
+    for _ in range(2):
+        sets.append(dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+                         qz=sa3.empty_quantized(B, H, N, d, dev), ws=torch.empty_like(ws),
+                         out=torch.empty_like(out),
+                         out_h=torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory(),
+                         ready=torch.cuda.Event(), done=torch.cuda.Event(), free=torch.cuda.Event()))
 
-    def e2e_step():
-        qd.copy_(qp, non_blocking=True)
-        kd.copy_(kp, non_blocking=True)
-        vd.copy_(vp, non_blocking=True)
-        sa3.quantize_qkv(qd, kd, vd, out=qz, workspace=ws)
-        sa3.attn_fwd(qz, causal=causal, out=out)
-        out_h.copy_(out, non_blocking=True)
+    def e2e_run(n):
+        for i in range(n):
+            b = sets[i % 2]
+            if i >= 2:
+                up_s.wait_event(b["free"])      # step i-2 has consumed and returned this set
+            with torch.cuda.stream(up_s):
+                b["q"].copy_(qp, non_blocking=True)
+                b["k"].copy_(kp, non_blocking=True)
+                b["v"].copy_(vp, non_blocking=True)
+                b["ready"].record(up_s)
+            stream.wait_event(b["ready"])
+            sa3.quantize_qkv(b["q"], b["k"], b["v"], out=b["qz"], workspace=b["ws"], stream=stream)
+            sa3.attn_fwd(b["qz"], causal=causal, out=b["out"], stream=stream)
+            b["done"].record(stream)
+            down_s.wait_event(b["done"])
+            with torch.cuda.stream(down_s):
+                b["out_h"].copy_(b["out"], non_blocking=True)
+                b["free"].record(down_s)
+        stream.wait_stream(up_s)
+        stream.wait_stream(down_s)
 
-    for _ in range(max(1, args.warmup // 2)):
-        e2e_step()
+    e2e_run(max(2, args.warmup // 2))
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = max(3, args.steps // 2)
     if world > 1:
         torch.distributed.barrier()
     e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
+    e2e_run(n_e2e)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if not torch.equal(sets[(n_e2e - 1) % 2]["out_h"], out.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident run")
 
     def gmax(x):
         if world == 1:
@@ -291,6 +314,7 @@ def run_sa3(args, rank, world, local):
                      "kernel": "attn_fwd_kernel<128>",
                      "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"},
         "e2e": {"value": round(world * ops / (t_e2e * 1e-3) / 1e12, 2), "unit": UNIT, "ms": round(t_e2e, 4),
+                "pipelined": "2 buffer sets; upload, kernels and download on three streams",
                 "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 2},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
