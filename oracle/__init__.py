@@ -13,6 +13,8 @@ Functions follow the method's steps in order:
   quantize_qkv     E2M1 codes + E4M3 scales per 16-element block
   attn_fwd         tiled online-softmax attention on the quantized operands
   attn_exact       fp64 softmax attention on the bf16 inputs (no quantization)
+  quantize_qkv_i8,
+  attn_fwd_i8      the 8-bit variant: INT8 Q, K per 128-token block, FP16 P, V
 Layouts are the canonical ones documented in ``sa3_oracle.c``.
 """
 from __future__ import annotations
@@ -77,6 +79,12 @@ def _load():
         lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, I, F, I, P, P, I, P]
         lib.oracle_attn_exact.restype = None
         lib.oracle_attn_exact.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, I, P]
+        lib.oracle_f32_to_f16.restype = ctypes.c_uint16
+        lib.oracle_f32_to_f16.argtypes = [F]
+        lib.oracle_quantize_qkv_i8.restype = None
+        lib.oracle_quantize_qkv_i8.argtypes = [P, P, P, I, I, I, I, I] + [P] * 6
+        lib.oracle_attn_fwd_i8.restype = None
+        lib.oracle_attn_fwd_i8.argtypes = [P] * 5 + [I, I, I, I, I, I, F, P, I, P]
         lib.oracle_num_threads.restype = I
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -219,6 +227,45 @@ def attn_exact(q, k, v, causal: bool, sm_scale: float | None = None,
     u, nu = _units_arr(units)
     _load().oracle_attn_exact(_ptr(q), _ptr(k), _ptr(v), B, H, N, Nkv, d, int(bool(causal)),
                               float(sm_scale), _ptr(k_sub), _ptr(u), nu, _ptr(out))
+    return out
+
+
+def f32_to_f16(x: float) -> int:
+    return _load().oracle_f32_to_f16(x)
+
+
+def quantize_qkv_i8(q, k, v) -> dict:
+    """8-bit variant (readings I1, I2): q_i8 [B,H,Np(Nq),d] int8, q_scale
+    [B,H,Np(Nq)/128] fp32 (one per 128-token block), k_i8 / k_scale the same
+    over Np(Nkv) after K smoothing, vt_f16 [B,H,d,Np(Nkv)] fp16 bits (uint16),
+    k_mean [B,H,d]; lengths n_q, n_kv."""
+    q, k, v = _as_u16(q), _as_u16(k), _as_u16(v)
+    B, H, Nq, d = q.shape
+    N = k.shape[2]
+    Npq, Np = padded_len(Nq), padded_len(N)
+    r = dict(q_i8=np.zeros((B, H, Npq, d), np.int8), q_scale=np.zeros((B, H, Npq // BLK), np.float32),
+             k_i8=np.zeros((B, H, Np, d), np.int8), k_scale=np.zeros((B, H, Np // BLK), np.float32),
+             vt_f16=np.zeros((B, H, d, Np), np.uint16), k_mean=np.zeros((B, H, d), np.float32))
+    _load().oracle_quantize_qkv_i8(_ptr(q), _ptr(k), _ptr(v), B, H, Nq, N, d, _ptr(r["q_i8"]), _ptr(r["q_scale"]),
+                                   _ptr(r["k_i8"]), _ptr(r["k_scale"]), _ptr(r["vt_f16"]), _ptr(r["k_mean"]))
+    r["n_q"], r["n_kv"] = Nq, N
+    return r
+
+
+def attn_fwd_i8(qz: dict, N: int, causal: bool, sm_scale: float | None = None, units=None,
+                n_kv: int | None = None) -> np.ndarray:
+    """8-bit variant attention (readings I3-I5) on quantize_qkv_i8 operands;
+    N query rows, n_kv keys (default qz["n_kv"] or N); bf16 bits [B,H,N,d]."""
+    if n_kv is None:
+        n_kv = qz.get("n_kv", N)
+    B, H, _, d = qz["q_i8"].shape
+    if sm_scale is None:
+        sm_scale = 1.0 / float(np.sqrt(d))
+    out = np.zeros((B, H, N, d), np.uint16)
+    u, nu = _units_arr(units)
+    arrs = [np.ascontiguousarray(qz[n]) for n in ("q_i8", "q_scale", "k_i8", "k_scale", "vt_f16")]
+    _load().oracle_attn_fwd_i8(*[_ptr(a) for a in arrs], B, H, N, n_kv, d, int(bool(causal)), float(sm_scale),
+                               _ptr(u), nu, _ptr(out))
     return out
 
 

@@ -473,6 +473,186 @@ void oracle_attn_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
 }
 
+/* ===================================================== 8-bit variant
+ * "SageAttention: Accurate 8-Bit Attention for Plug-and-play Inference
+ * Acceleration" (summary, "Approach"): Q and K quantized to INT8 with
+ * per-block scales after K is smoothed; P and V kept in FP16.  Readings
+ * (I1-I5, where the summary is silent):
+ *  I1 a block is one 128-token tile of Q or of K (the tiling above) over all
+ *     d channels: s = fp32(amax / 127), r = fp32(1 / s), code =
+ *     clamp(round_half_even(fp32(x * r)), -127, 127); s == 0 gives codes 0;
+ *  I2 V is converted to FP16 (round to nearest even), stored transposed;
+ *  I3 t = fp32(fp32(S) * f) with S the exact integer dot product and
+ *     f = fp32(fp32(s_q * s_k) * c), c = fp32(sm_scale * log2 e);
+ *  I4 P = exp2(t - m') as in R8, converted to FP16 (nearest even) before
+ *     P V; the row sum l accumulates the fp32 P;
+ *  I5 O accumulates in fp32 (the summary's ablation finds an FP16
+ *     accumulator changes nothing; fp32 is the tensor core's native one).
+ * Masks, lengths and the empty-row rule are those of R9, R11, R12. */
+
+/* fp32 -> fp16 bits, round to nearest even, overflow to inf. */
+uint16_t oracle_f32_to_f16(float x)
+{
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    double a = fabs((double)x);
+    if (isnan(x)) return (uint16_t)(sign | 0x7E00u);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                          /* a = m * 2^e, m in [0.5, 1) */
+    int qexp = (e - 1 >= -14) ? e - 11 : -24;  /* ulp: 10 fraction bits, or the subnormal step */
+    double v = nearbyint(ldexp(a, -qexp));  /* ties to even (default rounding mode) */
+    v = ldexp(v, qexp);
+    if (v > 65504.0) return (uint16_t)(sign | 0x7C00u);
+    if (v < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)ldexp(v, 24));  /* subnormal */
+    frexp(v, &e);
+    int ex = e - 1;                        /* v = 1.f * 2^ex */
+    uint16_t frac = (uint16_t)(ldexp(v, -ex) * 1024.0 - 1024.0);
+    return (uint16_t)(sign | ((uint16_t)(ex + 15) << 10) | frac);
+}
+
+static float f16_to_f32(uint16_t h)
+{
+    int ex = (h >> 10) & 31, fr = h & 1023;
+    double v = ex == 0 ? ldexp((double)fr, -24) : ldexp(1024.0 + fr, ex - 25);
+    if (ex == 31) v = fr ? NAN : INFINITY;
+    return (float)((h & 0x8000u) ? -v : v);
+}
+
+/* INT8 codes of n values with one scale (I1); returns the scale. */
+static float quant_block_i8(const float *x, int n, int8_t *codes)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float s = amax / 127.0f;
+    if (s == 0.0f) {
+        for (int i = 0; i < n; ++i) codes[i] = 0;
+        return 0.0f;
+    }
+    float r = 1.0f / s;
+    for (int i = 0; i < n; ++i) {
+        float y = x[i] * r;
+        float c = nearbyintf(y);
+        if (c > 127.0f) c = 127.0f;
+        if (c < -127.0f) c = -127.0f;
+        codes[i] = (int8_t)c;
+    }
+    return s;
+}
+
+/* Layouts: q_i8 [B*H][Np(Nq)][d], q_scale [B*H][Np(Nq)/128] fp32; k_i8,
+ * k_scale the same over Np(Nkv); vt_f16 [B*H][d][Np(Nkv)] fp16 bits;
+ * k_mean [B*H][d].  Padding tokens: code 0, fp16 0. */
+void oracle_quantize_qkv_i8(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            int B, int H, int Nq, int Nkv, int d,
+                            int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                            uint16_t *vt_f16, float *k_mean)
+{
+    const long BH = (long)B * H;
+    const int Npq = oracle_padded_len(Nq), Np = oracle_padded_len(Nkv);
+    oracle_kmean(k, B, H, Nkv, d, k_mean);
+    memset(q_i8, 0, (size_t)BH * Npq * d);
+    memset(k_i8, 0, (size_t)BH * Np * d);
+    memset(vt_f16, 0, (size_t)BH * d * Np * 2);
+#pragma omp parallel for schedule(dynamic)
+    for (long bh = 0; bh < BH; ++bh) {
+        float *x = (float *)malloc(sizeof(float) * BLK * d);
+        for (int which = 0; which < 2; ++which) {
+            const uint16_t *src = which ? k : q;
+            const int N = which ? Nkv : Nq, Npx = which ? Np : Npq;
+            int8_t *codes = which ? k_i8 : q_i8;
+            float *scale = which ? k_scale : q_scale;
+            for (int tb = 0; tb < Npx / BLK; ++tb) {
+                int n = 0;
+                for (int t = tb * BLK; t < tb * BLK + BLK && t < N; ++t)
+                    for (int c = 0; c < d; ++c) {
+                        float xv = bf16_to_f32(src[(bh * N + t) * d + c]);
+                        x[n++] = which ? xv - k_mean[bh * d + c] : xv;  /* K smoothed (R2) */
+                    }
+                scale[bh * (Npx / BLK) + tb] = quant_block_i8(x, n, codes + (bh * Npx + (long)tb * BLK) * d);
+            }
+        }
+        for (int c = 0; c < d; ++c)
+            for (int t = 0; t < Nkv; ++t)
+                vt_f16[(bh * d + c) * Np + t] = oracle_f32_to_f16(bf16_to_f32(v[(bh * Nkv + t) * d + c]));
+        free(x);
+    }
+}
+
+void oracle_attn_fwd_i8(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8, const float *k_scale,
+                        const uint16_t *vt_f16, int B, int H, int Nq, int Nkv, int d, int causal,
+                        float sm_scale, const int32_t *units, int n_units, uint16_t *out)
+{
+    const long BH = (long)B * H;
+    const int Npq = oracle_padded_len(Nq), Np = oracle_padded_len(Nkv);
+    const int nqb = Npq / BLK, off = Nkv - Nq;
+    const float c_log2 = (float)((double)sm_scale * 1.4426950408889634);
+    const long total = units ? n_units : BH * nqb;
+
+#pragma omp parallel for schedule(dynamic)
+    for (long u = 0; u < total; ++u) {
+        long bh = units ? units[2 * u] : u / nqb;
+        int qb = units ? units[2 * u + 1] : (int)(u % nqb);
+        int nkv = Np / BLK;
+        if (causal) {
+            int last = qb * BLK + BLK - 1 + off;
+            int nb = last < 0 ? 0 : last / BLK + 1;
+            if (nb < nkv) nkv = nb;
+        }
+        float *O = (float *)malloc(sizeof(float) * d);
+        /* FP16 V of this (batch, head), decoded once */
+        float *vhat = (float *)malloc(sizeof(float) * ((size_t)d * nkv * BLK + 1));
+        for (int c = 0; c < d; ++c)
+            for (int col = 0; col < nkv * BLK; ++col)
+                vhat[(size_t)c * nkv * BLK + col] = f16_to_f32(vt_f16[(bh * d + c) * Np + col]);
+        float t[BLK], p[BLK], p16[BLK];
+        for (int row = qb * BLK; row < qb * BLK + BLK && row < Nq; ++row) {
+            const int8_t *qr = q_i8 + (bh * Npq + row) * d;
+            float m = -INFINITY, l = 0.0f;
+            for (int c = 0; c < d; ++c) O[c] = 0.0f;
+            for (int j = 0; j < nkv; ++j) {
+                const float f = (q_scale[bh * nqb + qb] * k_scale[bh * (Np / BLK) + j]) * c_log2;  /* I3 */
+                float bmax = -INFINITY;
+                for (int i = 0; i < BLK; ++i) {
+                    int col = j * BLK + i;
+                    if (col >= Nkv || (causal && col > row + off)) { t[i] = -INFINITY; continue; }
+                    const int8_t *kr = k_i8 + (bh * Np + col) * d;
+                    long acc = 0;
+                    for (int c = 0; c < d; ++c) acc += (long)qr[c] * kr[c];
+                    t[i] = (float)acc * f;
+                    if (t[i] > bmax) bmax = t[i];
+                }
+                float m_new = m > bmax ? m : bmax;
+                float alpha;
+                if (m_new == -INFINITY) {
+                    alpha = 1.0f;
+                    for (int i = 0; i < BLK; ++i) p[i] = 0.0f;
+                } else {
+                    alpha = exp2f(m - m_new);
+                    for (int i = 0; i < BLK; ++i) p[i] = exp2f(t[i] - m_new);
+                }
+                double psum = 0.0;
+                for (int i = 0; i < BLK; ++i) psum += p[i];
+                l = alpha * l + (float)psum;
+                for (int i = 0; i < BLK; ++i) p16[i] = f16_to_f32(oracle_f32_to_f16(p[i]));  /* I4 */
+                for (int c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (int i = 0; i < BLK; ++i)
+                        acc += (double)p16[i] * (double)vhat[(size_t)c * nkv * BLK + j * BLK + i];
+                    O[c] = alpha * O[c] + (float)acc;
+                }
+                m = m_new;
+            }
+            for (int c = 0; c < d; ++c)
+                out[(bh * Nq + row) * d + c] = l > 0.0f ? oracle_f32_to_bf16(O[c] / l) : 0;
+        }
+        free(O);
+        free(vhat);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
