@@ -46,6 +46,11 @@ class _QKV(ctypes.Structure):
                 ("k_mean", ctypes.c_void_p)]
 
 
+class _QKVI8(ctypes.Structure):
+    _fields_ = [("q_i8", ctypes.c_void_p), ("q_scale", ctypes.c_void_p), ("k_i8", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p), ("vt_f16", ctypes.c_void_p), ("k_mean", ctypes.c_void_p)]
+
+
 _lock = threading.Lock()
 _lib = None
 
@@ -70,6 +75,10 @@ def lib() -> ctypes.CDLL:
             L.sa3_quantize_qkv_lens.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(_QKV), P, ctypes.c_size_t, P]
             L.sa3_attn_fwd_lens.restype = I
             L.sa3_attn_fwd_lens.argtypes = [ctypes.POINTER(_QKV), I, I, I, I, I, I, F, ctypes.c_uint, P, P]
+            L.sa3_quantize_qkv_i8.restype = I
+            L.sa3_quantize_qkv_i8.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(_QKVI8), P, ctypes.c_size_t, P]
+            L.sa3_attn_fwd_i8.restype = I
+            L.sa3_attn_fwd_i8.argtypes = [ctypes.POINTER(_QKVI8), I, I, I, I, I, I, F, P, P]
             L.sa3_device_status.restype = I
             L.sa3_device_status.argtypes = [P]
             _lib = L
@@ -199,6 +208,78 @@ def attn_fwd(qz: QuantizedQKV, causal: bool = False, sm_scale: float | None = No
                                      flags, out.data_ptr(), _stream_ptr(stream))
     if rc != SA3_OK:
         raise Sa3Error(rc, "sa3_attn_fwd")
+    return out
+
+
+# ------------------------------------------------------- 8-bit variant
+@dataclasses.dataclass
+class QuantizedQKVI8:
+    """Operands of the 8-bit variant (layouts: include/sa3.h): INT8 Q and
+    smoothed K with one fp32 scale per 128-token tile, FP16 V^T."""
+    q_i8: torch.Tensor     # int8 [B,H,Np(Nq),d]
+    q_scale: torch.Tensor  # f32 [B,H,Np(Nq)/128]
+    k_i8: torch.Tensor     # int8 [B,H,Np(N),d]
+    k_scale: torch.Tensor  # f32 [B,H,Np(N)/128]
+    vt_f16: torch.Tensor   # f16 [B,H,d,Np(N)]
+    k_mean: torch.Tensor   # f32 [B,H,d]
+    B: int
+    H: int
+    N: int
+    d: int
+    Nq: int
+
+    def struct(self) -> _QKVI8:
+        return _QKVI8(self.q_i8.data_ptr(), self.q_scale.data_ptr(), self.k_i8.data_ptr(), self.k_scale.data_ptr(),
+                      self.vt_f16.data_ptr(), self.k_mean.data_ptr())
+
+
+def empty_quantized_i8(B: int, H: int, N: int, d: int, device="cuda", Nq: int | None = None) -> QuantizedQKVI8:
+    Nq = N if Nq is None else Nq
+    Npq, Np = padded_len(Nq), padded_len(N)
+    f32 = dict(dtype=torch.float32, device=device)
+    return QuantizedQKVI8(
+        q_i8=torch.empty((B, H, Npq, d), dtype=torch.int8, device=device), q_scale=torch.empty((B, H, Npq // BLK), **f32),
+        k_i8=torch.empty((B, H, Np, d), dtype=torch.int8, device=device), k_scale=torch.empty((B, H, Np // BLK), **f32),
+        vt_f16=torch.empty((B, H, d, Np), dtype=torch.float16, device=device), k_mean=torch.empty((B, H, d), **f32),
+        B=B, H=H, N=N, d=d, Nq=Nq)
+
+
+def quantize_qkv_i8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: QuantizedQKVI8 | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> QuantizedQKVI8:
+    """sa3_quantize_qkv_i8: K smoothing, INT8 Q and K per 128-token tile, FP16 V^T."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_input(t, n)
+    if not (k.shape == v.shape and q.shape[:2] == k.shape[:2] and q.shape[3] == k.shape[3]):
+        raise ValueError("q must be [B,H,Nq,d] and k, v [B,H,N,d]")
+    B, H, Nq, d = q.shape
+    N = k.shape[2]
+    if out is None:
+        out = empty_quantized_i8(B, H, N, d, q.device, Nq=Nq)
+    if out.Nq != Nq or out.N != N:
+        raise ValueError("out was sized for other lengths")
+    if workspace is None:
+        workspace = torch.empty(max(quant_workspace_bytes(B, H, N, d), 16), dtype=torch.uint8, device=q.device)
+    st = out.struct()
+    rc = lib().sa3_quantize_qkv_i8(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, Nq, N, d, ctypes.byref(st),
+                                   workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if rc != SA3_OK:
+        raise Sa3Error(rc, "sa3_quantize_qkv_i8")
+    return out
+
+
+def attn_fwd_i8(qz: QuantizedQKVI8, causal: bool = False, sm_scale: float | None = None,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """sa3_attn_fwd_i8: 8-bit attention (INT8 QK^T, FP16 P V); bf16 [B,H,Nq,d]."""
+    B, H, N, d, Nq = qz.B, qz.H, qz.N, qz.d, qz.Nq
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=qz.q_i8.device)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    st = qz.struct()
+    rc = lib().sa3_attn_fwd_i8(ctypes.byref(st), B, H, Nq, N, d, int(bool(causal)), float(sm_scale),
+                               out.data_ptr(), _stream_ptr(stream))
+    if rc != SA3_OK:
+        raise Sa3Error(rc, "sa3_attn_fwd_i8")
     return out
 
 

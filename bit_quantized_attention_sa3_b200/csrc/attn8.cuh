@@ -1,0 +1,490 @@
+// attn8.cuh -- the 8-bit variant of the attention forward for sm_100a.
+//
+// Method ("SageAttention: Accurate 8-Bit Attention for Plug-and-play
+// Inference Acceleration", summary, "Approach"): Q and smoothed K in INT8
+// with per-block scales, P and V in FP16.  Per 128-row Q tile and 128-key
+// block j:
+//   S = Q8 K8_j^T                       tcgen05.mma kind::i8, int32 in TMEM
+//   t = S * f_j, f_j = fp32(fp32(s_q s_k,j) c)   (exact integer S)
+//   m' = max(m, rowmax t), alpha = 2^(m - m'), P = 2^(t - m'),
+//   l = alpha l + rowsum P, P16 = fp16(P)
+//   O = alpha O + P16 V16_j             tcgen05.mma kind::f16, fp32 in TMEM
+// and out = bf16(O / l).
+//
+// Same CTA organisation as the FP4 kernel (attn.cuh): two Q tiles per CTA,
+// 16 softmax warps (two threads per row, exchanging partial row maxima),
+// one TMA producer warp, one MMA-issuing warp; S in TMEM shared by the two
+// tiles.  Differences: no block-scale factors (so no tcgen05.cp and no
+// scale columns in TMEM); S is int32 and becomes fp32 exactly through the
+// 1.5 * 2^23 bias trick (|S| <= 127 * 127 * 128 < 2^22); P is 16 bits, so a
+// P tile is two 64-key 128-byte-swizzled atoms (32 KB) and a V^T tile two
+// 64-key atoms of d rows; two KV stages at d = 128 (three at d = 64).
+#pragma once
+
+#include "attn.cuh"
+
+namespace sa3 {
+namespace attn8 {
+
+using attn::drain_wait;
+using attn::ex2;
+using attn::kBlk;
+using attn::kSoftmaxWarps;
+using attn::kThreads;
+using attn::kWarpMma;
+using attn::kWarpProducer;
+using attn::max3f;
+using attn::warp_wait;
+
+template <int D>
+struct Cfg {
+    static constexpr int al(int x) { return (x + 1023) & ~1023; }
+    static constexpr int kStages = D == 128 ? 2 : 3;
+    static constexpr int kQBytes = kBlk * D;               // int8 Q or K tile: 128 rows x D bytes
+    static constexpr int kAtomBytes = kBlk * 128;          // 128 rows x 64 halves
+    static constexpr int kVAtomBytes = D * 128;            // D rows x 64 halves
+    static constexpr int kVBytes = 2 * kVAtomBytes;        // V^T tile: D rows x 128 keys
+    static constexpr int kPBytes = 2 * kAtomBytes;         // P tile: 128 rows x 128 keys
+    static constexpr uint32_t kQKLayout = D == 128 ? 2u : 4u;  // 128B / 64B swizzle
+    static constexpr uint32_t kQKSbo = 8 * D;
+    // shared memory map, offsets from a 1024-byte aligned base
+    static constexpr int oQ0 = 0;
+    static constexpr int oQ1 = al(oQ0 + kQBytes);
+    static constexpr int oStage = al(oQ1 + kQBytes);
+    static constexpr int sK = 0;
+    static constexpr int sV = al(kQBytes);
+    static constexpr int kStageBytes = al(sV + kVBytes);
+    static constexpr int oP0 = oStage + kStages * kStageBytes;
+    static constexpr int oP1 = oP0 + kPBytes;
+    static constexpr int oXch = oP1 + kPBytes;             // row maxima [2 parity][2 tiles][2 halves][128]
+    static constexpr int oXl = oXch + 4096;                // row sums [2 tiles][2 halves][128]
+    static constexpr int oBar = oXl + 2048;
+    static constexpr int kSmemBytes = oBar + 256 + 1024;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    // TMEM columns
+    static constexpr uint32_t tS = 0;
+    static constexpr uint32_t tO0 = 128;
+    static constexpr uint32_t tO1 = 128 + D;
+    static constexpr uint32_t kTmemCols = 512;
+};
+
+constexpr int kMaxStages = 3;
+enum : int {
+    kBarQ = 0,
+    kBarKvFull = 1,                    // kMaxStages
+    kBarKvEmpty = 1 + kMaxStages,      // kMaxStages
+    kBarSFull = 1 + 2 * kMaxStages,    // 2
+    kBarSEmpty = 3 + 2 * kMaxStages,   // 1
+    kBarPFull = 4 + 2 * kMaxStages,    // 2
+    kBarPvDone = 6 + 2 * kMaxStages,   // 2
+    kBarDrain = 8 + 2 * kMaxStages,    // 1
+    kBarXch = 9 + 2 * kMaxStages,      // 8
+    kBarCount = 17 + 2 * kMaxStages
+};
+static_assert(kBarCount * 8 + 8 <= 256, "barrier area");
+
+// Instruction descriptors (dense, K-major A and B, M = 128):
+// kind::i8: signed int8 A and B, int32 D;  kind::f16: f16 A and B, f32 D.
+__host__ __device__ constexpr uint32_t idesc_i8(int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (8u << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_f16(int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (8u << 24);
+}
+
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// int32 (|x| < 2^22) -> fp32, exactly, on the integer and FMA pipes.
+__device__ __forceinline__ float i2f_exact(uint32_t x) {
+    return __fsub_rn(__uint_as_float(x + 0x4B400000u), 12582912.0f);
+}
+
+// Two fp32 -> packed fp16x2 (round to nearest even), low half from `lo`.
+__device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <int D, bool kCross>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn8_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    using C = Cfg<D>;
+    constexpr int kStages = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t *base = smem_raw + (base_s - raw_s);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + C::oBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kBarCount);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // work units as in the FP4 kernel: pairs of Q tiles, then single tiles
+    const int nqt = p.Npq / kBlk;
+    const int nkvt = p.Np / kBlk;
+    const int off = kCross ? p.N - p.Nq : 0;
+    const int u = static_cast<int>(blockIdx.x);
+    const bool single = u >= p.pair_units;
+    const int pu = single ? p.pair_units + (u - p.pair_units) / 2 : u;
+    const int bh = pu % p.BH;
+    const int rank = pu / p.BH;
+    const int pair = p.causal ? p.npairs - 1 - rank : rank;
+    const int tile0 = 2 * pair + (single ? ((u - p.pair_units) & 1) : 0);
+    const int tile1 = tile0 + 1;
+    if (tile0 >= nqt) return;
+    const bool valid1 = !single && tile1 < nqt;
+    auto n_blocks = [&](int tile) -> int {
+        if (!p.causal) return nkvt;
+        const int last = tile * kBlk + kBlk - 1 + off;
+        const int nb = last < 0 ? 0 : last / kBlk + 1;
+        return nb < nkvt ? nb : nkvt;
+    };
+    const int n0 = n_blocks(tile0);
+    const int n1 = valid1 ? n_blocks(tile1) : 0;
+    const int nmax = n0 > n1 ? n0 : n1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars + kBarQ, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bars + kBarKvFull + s, 1);
+            mbar_init(bars + kBarKvEmpty + s, 1);
+        }
+        mbar_init(bars + kBarSFull + 0, 1);
+        mbar_init(bars + kBarSFull + 1, 1);
+        mbar_init(bars + kBarSEmpty, 256);
+        mbar_init(bars + kBarPFull + 0, 256);
+        mbar_init(bars + kBarPFull + 1, 256);
+        mbar_init(bars + kBarPvDone + 0, 1);
+        mbar_init(bars + kBarPvDone + 1, 1);
+        mbar_init(bars + kBarDrain, 1);
+        for (int x = 0; x < 8; ++x) mbar_init(bars + kBarXch + x, 64);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= kWarpProducer) {
+      if (warp == kWarpProducer) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            uint64_t *bq = bars + kBarQ;
+            mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * C::kQBytes);
+            tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Npq + tile0 * kBlk, bq);
+            if (valid1) tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Npq + tile1 * kBlk, bq);
+            int issued = 0;
+            for (int j = 0; j < nmax; ++j) {
+                const int s = j % kStages;
+                const int r = j / kStages;
+                if (r > 0 && !mbar_wait(bars + kBarKvEmpty + s, (r - 1) & 1, abort_flag)) break;
+                uint8_t *st = base + C::oStage + s * C::kStageBytes;
+                uint64_t *bf = bars + kBarKvFull + s;
+                mbar_arrive_expect_tx(bf, C::kQBytes + C::kVBytes);
+                tma_load_2d(st + C::sK, &tm_k, 0, bh * p.Np + j * kBlk, bf);
+                // V^T: keys 64a .. 64a+63 of block j for every channel, two 128-byte-wide boxes
+                tma_load_2d(st + C::sV, &tm_v, j * 256, bh * D, bf);
+                tma_load_2d(st + C::sV + C::kVAtomBytes, &tm_v, j * 256 + 128, bh * D, bf);
+                issued = j + 1;
+            }
+            drain_wait(bq, 0);
+            for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
+                drain_wait(bars + kBarKvFull + j % kStages, (j / kStages) & 1);
+        }
+    } else {
+        // ----------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t kIdQK = idesc_i8(128);
+            constexpr uint32_t kIdPV = idesc_f16(D);
+            int nqk = 0;
+            auto stage_s = [&](int j) -> uint32_t {
+                return base_s + C::oStage + static_cast<uint32_t>(j % kStages) * C::kStageBytes;
+            };
+            auto issue_qk = [&](int i, int j) -> bool {
+                if (nqk > 0 && !mbar_wait(bars + kBarSEmpty, (nqk - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t qa = base_s + (i ? C::oQ1 : C::oQ0);
+                const uint32_t kb = stage_s(j) + C::sK;
+#pragma unroll
+                for (int kc = 0; kc < D / 32; ++kc)  // K = 32 int8 per instruction
+                    tc_mma_i8(tmem + C::tS, sdesc_kmajor_sw(qa + 32 * kc, C::kQKSbo, C::kQKLayout),
+                              sdesc_kmajor_sw(kb + 32 * kc, C::kQKSbo, C::kQKLayout), kIdQK, kc > 0);
+                tc_commit(bars + kBarSFull + i);
+                ++nqk;
+                return true;
+            };
+            auto issue_pv = [&](int i, int j) -> bool {
+                if (!mbar_wait(bars + kBarPFull + i, j & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t pa = base_s + (i ? C::oP1 : C::oP0);
+                const uint32_t vb = stage_s(j) + C::sV;
+#pragma unroll
+                for (int kc = 0; kc < 8; ++kc) {  // K = 16 halves per instruction, 4 per 64-key atom
+                    const uint32_t a = pa + (kc >> 2) * C::kAtomBytes + 32 * (kc & 3);
+                    const uint32_t b = vb + (kc >> 2) * C::kVAtomBytes + 32 * (kc & 3);
+                    tc_mma_f16(tmem + (i ? C::tO1 : C::tO0), sdesc_kmajor_sw(a, 1024, 2u),
+                               sdesc_kmajor_sw(b, 1024, 2u), kIdPV, (j > 0 || kc > 0) ? 1u : 0u);
+                }
+                tc_commit(bars + kBarPvDone + i);
+                return true;
+            };
+
+            bool ok = mbar_wait(bars + kBarQ, 0, abort_flag);
+            if (ok && nmax > 0) ok = mbar_wait(bars + kBarKvFull + 0, 0, abort_flag);
+            if (ok && nmax > 0) {
+                tc_fence_after();
+                if (n0 > 0) ok = issue_qk(0, 0);
+                if (ok && n1 > 0) ok = issue_qk(1, 0);
+            }
+            for (int j = 0; ok && j < nmax; ++j) {
+                if (j + 1 < nmax) {
+                    ok = mbar_wait(bars + kBarKvFull + (j + 1) % kStages, ((j + 1) / kStages) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                if (j + 1 < n0 && !(ok = issue_qk(0, j + 1))) break;
+                if (j < n0 && !(ok = issue_pv(0, j))) break;
+                if (j + 1 < n1 && !(ok = issue_qk(1, j + 1))) break;
+                if (j < n1 && !(ok = issue_pv(1, j))) break;
+                tc_commit(bars + kBarKvEmpty + j % kStages);
+            }
+            tc_commit(bars + kBarDrain);
+            drain_wait(bars + kBarDrain, 0);
+        }
+        __syncwarp();
+      }
+    } else {
+        // ------------------------------------------------------- softmax
+        // Warp w: Q tile w/8, column half (w/4)%2, TMEM lanes 32*(w%4)..:
+        // one row per thread, two threads per row (as in the FP4 kernel).
+        const int i = warp >> 3;
+        const int h = (warp >> 2) & 1;
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const int tile = i ? tile1 : tile0;
+        const int grow = tile * kBlk + r;
+        const int n_i = i ? n1 : n0;
+        uint64_t *xbar = bars + kBarXch + 4 * i + wq;
+        const float c2 = p.scale_log2;
+        const float sq = n_i > 0 ? p.q_scale[static_cast<size_t>(bh) * nqt + tile] : 0.0f;
+        const float *sk = p.k_scale + static_cast<size_t>(bh) * nkvt;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t tO = (i ? C::tO1 : C::tO0) + h * (D / 2);
+        // this half's 64 keys are P atom h: row r at (r/8)*1024 + (r%8)*128
+        uint8_t *prow = base + (i ? C::oP1 : C::oP0) + h * C::kAtomBytes + (r >> 3) * 1024 + (r & 7) * 128;
+        float *xch = reinterpret_cast<float *>(base + C::oXch);
+        float *xl = reinterpret_cast<float *>(base + C::oXl) + (i * 2) * kBlk;
+        float m = -INFINITY;
+        float l = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < n_i; ++j) {
+            if (!warp_wait(bars + kBarSFull + i, j & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t s[2][32];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) tmem_ld32(trow + C::tS + 64 * h + 32 * q, s[q]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) reg_fence32(s[q]);
+            tc_fence_before();
+            mbar_arrive(bars + kBarSEmpty);
+
+            // exact fp32 of the integer scores, in place
+#pragma unroll
+            for (int e = 0; e < 64; ++e) s[e >> 5][e & 31] = __float_as_uint(i2f_exact(s[e >> 5][e & 31]));
+            auto x = [&](int e) -> float { return __uint_as_float(s[e >> 5][e & 31]); };
+            const int col0 = j * kBlk + 64 * h;
+            const bool tail = col0 + 64 > p.N;
+            const bool diag = p.causal && (col0 + 63 > tile * kBlk + off);
+            if (tail || diag) {
+                int lim = p.N - col0;
+                if (p.causal) lim = min(lim, grow + off - col0 + 1);
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    if (e >= lim) s[e >> 5][e & 31] = __float_as_uint(-INFINITY);
+            }
+            // partial row maximum: four independent 3-input chains, then combined
+            float mx[4] = {x(0), x(1), x(2), x(3)};
+#pragma unroll
+            for (int e = 4; e < 64; e += 8) {
+                mx[0] = max3f(mx[0], x(e), x(e + 1));
+                mx[1] = max3f(mx[1], x(e + 2), x(e + 3));
+                mx[2] = max3f(mx[2], x(e + 4), x(e + 5));
+                mx[3] = max3f(mx[3], x(e + 6), x(e + 7));
+            }
+            float *xs = xch + (((j & 1) * 2 + i) * 2) * kBlk;
+            xs[h * kBlk + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            mbar_arrive(xbar);
+            if (!warp_wait(xbar, j & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const float rmax = fmaxf(xs[r], xs[kBlk + r]);
+            // t = S * f with f = fp32(fp32(s_q s_k) c) > 0 (floored at the
+            // smallest normal so that a zero block gives t = +-0, not 0 * inf)
+            const float f = fmaxf(__fmul_rn(__fmul_rn(sq, sk[j]), c2), 1.17549435e-38f);
+            const float tmax = rmax == -INFINITY ? -INFINITY : __fmul_rn(rmax, f);
+            const float m_new = kCross ? fmaxf(fmaxf(m, tmax), -3.402823466e38f) : fmaxf(m, tmax);
+            const float nm = -m_new;
+            const float alpha = ex2(__fsub_rn(m, m_new));
+            // P = 2^(t - m'), fp32 row sum, fp16 P for P V; written to shared
+            // memory in two halves of 32 keys (16-byte chunk c of this half,
+            // keys 8c .. 8c+7, at chunk c ^ (r % 8)), the first one once the
+            // previous P V has released the buffer
+            const uint64_t ff = pack2(f, f);
+            const uint64_t nn = pack2(nm, nm);
+            uint64_t acc = pack2(0.0f, 0.0f);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t ph[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int k = 32 * half + 2 * e;
+                    const uint64_t t2 = fma2(pack2(x(k), x(k + 1)), ff, nn);
+                    const float p0 = ex2(lo2(t2)), p1 = ex2(hi2(t2));
+                    acc = add2(acc, pack2(p0, p1));
+                    ph[e] = f16x2(p0, p1);
+                }
+                if (half == 0 && j > 0) {
+                    if (!warp_wait(bars + kBarPvDone + i, (j - 1) & 1, abort_flag)) ok = false;
+                    tc_fence_after();
+                }
+                if (ok) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int cc = 4 * half + c;
+                        *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) =
+                            make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+                    }
+                }
+            }
+            if (!ok) break;
+            l = alpha * l + (lo2(acc) + hi2(acc));
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                uint32_t o[D / 64][32];
+#pragma unroll
+                for (int q = 0; q < D / 64; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
+                tmem_ld_wait();
+                const uint64_t aa = pack2(alpha, alpha);
+#pragma unroll
+                for (int q = 0; q < D / 64; ++q) {
+                    reg_fence32(o[q]);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const uint64_t v = mul2(pack2(__uint_as_float(o[q][e]), __uint_as_float(o[q][e + 1])), aa);
+                        o[q][e] = __float_as_uint(lo2(v));
+                        o[q][e + 1] = __float_as_uint(hi2(v));
+                    }
+                    tmem_st32(trow + tO + 32 * q, o[q]);
+                }
+                tmem_st_wait();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bars + kBarPFull + i);
+            m = m_new;
+        }
+        float l_row = 0.0f;
+        if (ok && n_i > 0) {
+            xl[h * kBlk + r] = l;
+            mbar_arrive(xbar);
+            ok = warp_wait(xbar, n_i & 1, abort_flag);
+            l_row = xl[r] + xl[kBlk + r];
+        }
+        if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
+            tc_fence_after();
+            const float inv = (!kCross || l_row > 0.0f) ? __frcp_rn(l_row) : 0.0f;
+            __nv_bfloat16 *orow = p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2);
+#pragma unroll
+            for (int q = 0; q < D / 64; ++q) {
+                uint32_t o[32];
+                tmem_ld32(trow + tO + 32 * q, o);
+                tmem_ld_wait();
+                reg_fence32(o);
+                if (grow < p.Nq) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                                        __uint_as_float(o[2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * q);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                }
+            }
+        } else if (kCross && ok && n_i == 0 && i <= static_cast<int>(valid1) && grow < p.Nq) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2));
+#pragma unroll
+            for (int v = 0; v < D / 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     cudaStream_t stream) {
+    using C = Cfg<D>;
+    auto kernel = p.Nq != p.N ? attn8_fwd_kernel<D, true> : attn8_fwd_kernel<D, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    AttnParams q = p;
+    const int nqt = p.Npq / kBlk;
+    q.npairs = (nqt + 1) / 2;
+    const int total = q.npairs * p.BH;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int rem = total % nsm;
+    const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
+    q.pair_units = total - split;
+    kernel<<<dim3(q.pair_units + 2 * split), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
+    return cudaGetLastError();
+}
+
+}  // namespace attn8
+
+inline cudaError_t launch_attn_i8(const AttnParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                  const CUtensorMap &tm_v, int d, cudaStream_t stream) {
+    return d == 128 ? attn8::launch_d<128>(p, tm_q, tm_k, tm_v, stream)
+                    : attn8::launch_d<64>(p, tm_q, tm_k, tm_v, stream);
+}
+
+}  // namespace sa3

@@ -215,6 +215,101 @@ __device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int Np
     }
 }
 
+// ------------------------------------------------- 8-bit variant tiles
+// One staged 128-token tile of Q or K as INT8 with one scale for the whole
+// tile ("SageAttention" summary, "Approach"; per-block scales):
+// s = fp32(amax / 127), r = fp32(1 / s), code = clamp(rn_even(fp32(x r)),
+// +-127).  Thread: token row t/2, channel half t%2.  red: 8 floats of
+// shared scratch.  Returns nothing; thread 0 stores the scale.
+template <int D, bool kSmooth>
+__device__ __forceinline__ void qk_tile_i8(const uint8_t *__restrict__ stage, int N, int tile,
+                                           const float *__restrict__ neg_mean, int8_t *__restrict__ codes,
+                                           float *__restrict__ scale_out, float *red) {
+    constexpr int kCh = D / 2;  // channels per thread
+    const int row = static_cast<int>(threadIdx.x) >> 1;
+    const int part = static_cast<int>(threadIdx.x) & 1;
+    const int t = tile * kTile + row;
+    float x[kCh];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c8 = 0; c8 < kCh / 8; ++c8) {
+        const int ch0 = part * kCh + c8 * 8;
+        const uint4 w = *reinterpret_cast<const uint4 *>(stage + tile_off(row, ch0));
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[c8 * 8 + 2 * e] = bf16_lo(u[e]);
+            x[c8 * 8 + 2 * e + 1] = bf16_hi(u[e]);
+        }
+        if (kSmooth && t < N) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[c8 * 8 + e] = __fadd_rn(x[c8 * 8 + e], neg_mean[ch0 + e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[c8 * 8 + e]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    float a = red[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) a = fmaxf(a, red[w]);
+    const float s = __fdiv_rn(a, 127.0f);
+    const float r = s == 0.0f ? 0.0f : __frcp_rn(s);
+    uint32_t pk[kCh / 4];
+#pragma unroll
+    for (int i = 0; i < kCh / 4; ++i) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int c = __float2int_rn(__fmul_rn(x[4 * i + e], r));  // round half to even
+            c = c > 127 ? 127 : (c < -127 ? -127 : c);
+            word |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * e);
+        }
+        pk[i] = word;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(codes + static_cast<size_t>(t) * D + part * kCh);
+#pragma unroll
+    for (int i = 0; i < kCh / 16; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    if (threadIdx.x == 0) scale_out[tile] = s;
+    __syncthreads();  // red is rewritten by the next tile
+}
+
+// One staged 128-token tile of V as FP16 (round to nearest even), stored
+// transposed: vt [d][Np] halves.  Thread: channel pair (2cp, 2cp+1),
+// 16-token blocks g*D/64 .. g*D/64 + D/64 - 1, one 32-byte row piece per
+// channel and block.
+template <int D>
+__device__ __forceinline__ void v_tile_f16(const uint8_t *__restrict__ stage, int Np, int tile,
+                                           uint8_t *__restrict__ vt) {
+    constexpr int kPairs = D / 2;
+    constexpr int kTbpt = D / 64;
+    const int cp = static_cast<int>(threadIdx.x) % kPairs;
+    const int g = static_cast<int>(threadIdx.x) / kPairs;
+#pragma unroll
+    for (int i = 0; i < kTbpt; ++i) {
+        const int tb = g * kTbpt + i;
+        uint32_t h0[8], h1[8];
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+            const int r = tb * 16 + k;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(stage + tile_off(r, 2 * cp));
+            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(stage + tile_off(r + 1, 2 * cp));
+            const __half2 a = __floats2half2_rn(bf16_lo(w0), bf16_lo(w1));  // channel 2cp, tokens r, r+1
+            const __half2 b = __floats2half2_rn(bf16_hi(w0), bf16_hi(w1));  // channel 2cp+1
+            h0[k / 2] = *reinterpret_cast<const uint32_t *>(&a);
+            h1[k / 2] = *reinterpret_cast<const uint32_t *>(&b);
+        }
+        uint8_t *r0 = vt + (static_cast<size_t>(2 * cp) * Np + tile * kTile + tb * 16) * 2;
+        uint8_t *r1 = r0 + static_cast<size_t>(Np) * 2;
+        reinterpret_cast<uint4 *>(r0)[0] = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+        reinterpret_cast<uint4 *>(r0)[1] = make_uint4(h0[4], h0[5], h0[6], h0[7]);
+        reinterpret_cast<uint4 *>(r1)[0] = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+        reinterpret_cast<uint4 *>(r1)[1] = make_uint4(h1[4], h1[5], h1[6], h1[7]);
+    }
+}
+
 // fp64 column sums of one staged K tile into this thread's accumulators:
 // channels 8v .. 8v+7 of rows r0, r0 + kRowStep, ...
 template <int D>
@@ -397,7 +492,8 @@ __device__ __forceinline__ SmemPtrs smem_setup(uint8_t *raw) {
 
 // -------------------------------------------------------------- kernels
 // First launch: Q and V tiles, then fp64 column sums of K per chunk.
-template <int D>
+// kI8: the 8-bit variant (INT8 Q, K with one scale per tile; FP16 V).
+template <int D, bool kI8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     quant_qvk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const QuantParams p) {
@@ -435,12 +531,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         const uint8_t *st = sm.base + s * QCfg<D>::kTileBytes;
         if (t.kind == 0) {
-            qk_tile<D, false>(st, p.Nq, t.tile, nullptr, sm.lut,
-                              p.q_fp4 + static_cast<size_t>(t.bh) * p.Npq * (D / 2),
-                              p.q_sf + static_cast<size_t>(t.bh) * p.Npq * (D / 16));
+            if constexpr (kI8)
+                qk_tile_i8<D, false>(st, p.Nq, t.tile, nullptr,
+                                     reinterpret_cast<int8_t *>(p.q_fp4) + static_cast<size_t>(t.bh) * p.Npq * D,
+                                     p.q_scale + static_cast<size_t>(t.bh) * (p.Npq / kTile),
+                                     reinterpret_cast<float *>(sm.red));
+            else
+                qk_tile<D, false>(st, p.Nq, t.tile, nullptr, sm.lut,
+                                  p.q_fp4 + static_cast<size_t>(t.bh) * p.Npq * (D / 2),
+                                  p.q_sf + static_cast<size_t>(t.bh) * p.Npq * (D / 16));
         } else if (t.kind == 1) {
-            v_tile<D>(st, p.Np, t.tile, sm.lut, p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
-                      p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
+            if constexpr (kI8)
+                v_tile_f16<D>(st, p.Np, t.tile, p.vt_fp4 + static_cast<size_t>(t.bh) * D * p.Np * 2);
+            else
+                v_tile<D>(st, p.Np, t.tile, sm.lut, p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
+                          p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
         } else {
             ksum_tile<D>(st, acc);
         }
@@ -457,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // Second launch: K tiles [g*T/G, (g+1)*T/G) of the T = BH * ntile tiles,
 // smoothed by the mean of their (b, h) and quantized.
-template <int D>
+template <int D, bool kI8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     quant_k_kernel(const __grid_constant__ CUtensorMap tm_k, const QuantParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -509,9 +614,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             ok = false;
             break;
         }
-        qk_tile<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean, sm.lut,
-                         p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
-                         p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16));
+        if constexpr (kI8)
+            qk_tile_i8<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean,
+                                reinterpret_cast<int8_t *>(p.k_fp4) + static_cast<size_t>(bh) * p.Np * D,
+                                p.k_scale + static_cast<size_t>(bh) * (p.Np / kTile), reinterpret_cast<float *>(sm.red));
+        else
+            qk_tile<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean, sm.lut,
+                             p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
+                             p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16));
         __syncthreads();  // stage s and neg_mean have been read by every thread
         if (threadIdx.x == 0 && i0 + n + kStages < i1) {
             fence_proxy_async_smem();
@@ -523,15 +633,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (!ok && threadIdx.x == 0) ring_drain(sm.full, n, issued);
 }
 
-template <int D>
+template <int D, bool kI8>
 cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      cudaStream_t stream) {
     using C = QCfg<D>;
     if (p.nchunk > kMaxChunks || p.chunk % kTile != 0) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(quant_qvk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(quant_qvk_kernel<D, kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(quant_k_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(quant_k_kernel<D, kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -540,7 +650,7 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
                              static_cast<long long>(p.BH) * p.nchunk;
     const long long slots = static_cast<long long>(nsm) * kCtasPerSm;
     const int grid_a = static_cast<int>(work_a < slots ? work_a : slots);
-    quant_qvk_kernel<D><<<grid_a, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    quant_qvk_kernel<D, kI8><<<grid_a, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long tiles_k = p.BH * ntile;
@@ -554,7 +664,7 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quant_k_kernel<D>, tk, p);
+    return cudaLaunchKernelEx(&cfg, quant_k_kernel<D, kI8>, tk, p);
 }
 
 }  // namespace quant
@@ -564,7 +674,15 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
 // with 64 x 128 boxes and 128-byte swizzle.
 inline cudaError_t launch_quant(const QuantParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, int d, cudaStream_t stream) {
-    return d == 128 ? quant::launch_d<128>(p, tq, tk, tv, stream) : quant::launch_d<64>(p, tq, tk, tv, stream);
+    return d == 128 ? quant::launch_d<128, false>(p, tq, tk, tv, stream)
+                    : quant::launch_d<64, false>(p, tq, tk, tv, stream);
+}
+// The 8-bit variant: INT8 Q, K (one fp32 scale per 128-token tile, K
+// smoothed) and FP16 V^T, same schedule and launches.
+inline cudaError_t launch_quant_i8(const QuantParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                   const CUtensorMap &tv, int d, cudaStream_t stream) {
+    return d == 128 ? quant::launch_d<128, true>(p, tq, tk, tv, stream)
+                    : quant::launch_d<64, true>(p, tq, tk, tv, stream);
 }
 
 }  // namespace sa3

@@ -18,6 +18,7 @@
 #include "sm100.cuh"
 
 #include "attn.cuh"
+#include "attn8.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -164,6 +165,42 @@ int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, in
                                                                                                         : SA3_ERR_CUDA;
 }
 
+int sa3_quantize_qkv_i8(const void *q, const void *k, const void *v, int B, int H, int Nq, int Nkv, int d,
+                        const sa3_qkv_i8 *out, void *workspace, size_t workspace_bytes,
+                        struct CUstream_st *stream) {
+    int rc = check_shape(B, H, Nq, d);
+    if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
+    if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
+    if (!out || !out->q_i8 || !out->q_scale || !out->k_i8 || !out->k_scale || !out->vt_f16 || !out->k_mean ||
+        !aligned16(out->q_i8) || !aligned16(out->q_scale) || !aligned16(out->k_i8) || !aligned16(out->k_scale) ||
+        !aligned16(out->vt_f16) || !aligned16(out->k_mean))
+        return SA3_ERR_INVALID_ARG;
+    const int64_t need = sa3_quant_workspace_bytes(B, H, Nkv, d);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
+    sa3::QuantParams p = {};
+    p.q_fp4 = static_cast<uint8_t *>(out->q_i8);
+    p.k_fp4 = static_cast<uint8_t *>(out->k_i8);
+    p.vt_fp4 = static_cast<uint8_t *>(out->vt_f16);
+    p.q_scale = out->q_scale;
+    p.k_scale = out->k_scale;
+    p.k_mean = out->k_mean;
+    p.part = static_cast<double *>(workspace);
+    p.BH = B * H;
+    p.N = Nkv;
+    p.Np = static_cast<int>(sa3_padded_len(Nkv));
+    p.Nq = Nq;
+    p.Npq = static_cast<int>(sa3_padded_len(Nq));
+    p.chunk = static_cast<int>(sa3_kmean_chunk(Nkv));
+    p.nchunk = static_cast<int>(sa3_kmean_nchunk(Nkv));
+    CUtensorMap tq, tk, tv;
+    if (!make_qkv_map(&tq, q, d, Nq, p.BH) || !make_qkv_map(&tk, k, d, Nkv, p.BH) ||
+        !make_qkv_map(&tv, v, d, Nkv, p.BH))
+        return SA3_ERR_CUDA;
+    return sa3::launch_quant_i8(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA3_OK
+               : SA3_ERR_CUDA;
+}
+
 int sa3_quantize_qkv(const void *q, const void *k, const void *v, int B, int H, int N, int d,
                      const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes, struct CUstream_st *stream) {
     return sa3_quantize_qkv_lens(q, k, v, B, H, N, N, d, out, workspace, workspace_bytes, stream);
@@ -216,6 +253,42 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
     p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
     p.p_pre_log2 = (flags & SA3_P_TWO_LEVEL) ? 11.0f : 0.0f;
     return sa3::launch_attn(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA3_OK
+               : SA3_ERR_CUDA;
+}
+
+int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                    void *out, struct CUstream_st *stream) {
+    int rc = check_shape(B, H, Nq, d);
+    if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
+    if (!in || !in->q_i8 || !in->q_scale || !in->k_i8 || !in->k_scale || !in->vt_f16 || !aligned16(in->q_i8) ||
+        !aligned16(in->k_i8) || !aligned16(in->vt_f16))
+        return SA3_ERR_INVALID_ARG;
+    if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
+    if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
+    const int BH = B * H;
+    const int Npq = static_cast<int>(sa3_padded_len(Nq));
+    const int Np = static_cast<int>(sa3_padded_len(Nkv));
+    CUtensorMap tq, tk, tv;
+    const CUtensorMapSwizzle qk_sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!make_map(&tq, in->q_i8, d, static_cast<uint64_t>(BH) * Npq, d, 128, qk_sw) ||
+        !make_map(&tk, in->k_i8, d, static_cast<uint64_t>(BH) * Np, d, 128, qk_sw) ||
+        !make_map(&tv, in->vt_f16, static_cast<uint64_t>(Np) * 2, static_cast<uint64_t>(BH) * d, 128, d,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return SA3_ERR_CUDA;
+    sa3::AttnParams p = {};
+    p.q_scale = in->q_scale;
+    p.k_scale = in->k_scale;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.BH = BH;
+    p.N = Nkv;
+    p.Np = Np;
+    p.Nq = Nq;
+    p.Npq = Npq;
+    p.causal = causal;
+    p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+    return sa3::launch_attn_i8(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA3_OK
                : SA3_ERR_CUDA;
 }

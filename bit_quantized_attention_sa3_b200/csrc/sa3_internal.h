@@ -18,7 +18,9 @@ struct QuantParams {
     uint8_t *vt_fp4;
     uint8_t *vt_sf;
     float *k_mean;
-    double *part;  // [BH][nchunk][d] scratch: fp64 column sums of K per chunk
+    float *q_scale;  // 8-bit variant: one fp32 scale per 128-token tile of Q
+    float *k_scale;  // ... and of K (codes then go to q_fp4 / k_fp4 as int8, V to vt_fp4 as fp16)
+    double *part;    // [BH][nchunk][d] scratch: fp64 column sums of K per chunk
     int BH;
     int N;       // K and V tokens
     int Np;      // N rounded up to 128
@@ -32,6 +34,8 @@ struct AttnParams {
     const uint8_t *q_sf;
     const uint8_t *k_sf;
     const uint8_t *vt_sf;
+    const float *q_scale;  // 8-bit variant: fp32 scale per 128-token tile of Q
+    const float *k_scale;  // ... and of K
     __nv_bfloat16 *out;
     int BH;
     int N;             // key / value tokens

@@ -195,6 +195,49 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
                       struct CUstream_st *stream);
 
 /*
+ * 8-bit variant ("SageAttention: Accurate 8-Bit Attention for Plug-and-play
+ * Inference Acceleration", summary, "Approach"): Q and K quantized to INT8
+ * with per-block scales after K smoothing, P and V kept in FP16.  Blocks are
+ * the 128-token tiles of the FP4 path, taken over all d channels:
+ *   s = fp32(amax / 127), r = fp32(1 / s),
+ *   code = clamp(round_half_even(fp32(x * r)), -127, 127), all 0 if s == 0;
+ * V is converted to FP16 (nearest even).  Attention: S = integer dot of the
+ * codes (exact, int32 on the tensor cores), t = fp32(S) * fp32(fp32(s_q *
+ * s_k) * sm_scale * log2 e), the online softmax of sa3_attn_fwd, P
+ * converted to FP16, O += P V in fp32, out = bf16(O / l).  Lengths, masks
+ * and the empty-row rule as in sa3_attn_fwd_lens.  No E4M3 block scales.
+ *
+ *   q_i8     int8 [B*H][N_p(Nq)][d]       q_scale  fp32 [B*H][N_p(Nq)/128]
+ *   k_i8     int8 [B*H][N_p(Nkv)][d]      k_scale  fp32 [B*H][N_p(Nkv)/128]
+ *   vt_f16   fp16 [B*H][d][N_p(Nkv)]      k_mean   fp32 [B*H][d]
+ * Padding tokens: code 0, fp16 0.  All device pointers, 16-byte aligned.
+ */
+typedef struct sa3_qkv_i8 {
+    void *q_i8;
+    float *q_scale;
+    void *k_i8;
+    float *k_scale;
+    void *vt_f16;
+    float *k_mean;
+} sa3_qkv_i8;
+static inline int64_t sa3_i8_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ return B * H * sa3_padded_len(N) * d; }
+static inline int64_t sa3_i8_scale_bytes(int64_t B, int64_t H, int64_t N)
+{ return B * H * (sa3_padded_len(N) / 128) * 4; }
+static inline int64_t sa3_vt_f16_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
+{ return B * H * d * sa3_padded_len(N) * 2; }
+
+/* workspace: sa3_quant_workspace_bytes(B, H, Nkv, d), as for the FP4 path. */
+int sa3_quantize_qkv_i8(const void *q, const void *k, const void *v,
+                        int B, int H, int Nq, int Nkv, int d,
+                        const sa3_qkv_i8 *out,
+                        void *workspace, size_t workspace_bytes,
+                        struct CUstream_st *stream);
+int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d,
+                    int causal, float sm_scale, void *out,
+                    struct CUstream_st *stream);
+
+/*
  * sa3_quantize_qkv_noalloc -- sa3_quantize_qkv without a caller workspace.
  *
  * There is no counterpart in the paper: this is a convenience for callers
