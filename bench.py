@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sa3", choices=["sa3", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=list(sa3_inputs.WORKLOADS))
+    ap.add_argument("--variant", default="fp4", choices=["fp4", "i8"],
+                    help="fp4: the microscaled FP4 path (the headline); i8: the 8-bit variant "
+                         "(INT8 QK^T, FP16 P V)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
     return ap.parse_args()
@@ -174,7 +177,11 @@ def run_sa3(args, rank, world, local):
     B, H, N, d, causal = w.B, w.H, w.N, w.d, w.causal
     q_h, k_h, v_h = sa3_inputs.make_qkv(w, seed=rank)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    qz = sa3.empty_quantized(B, H, N, d, dev)
+    i8 = args.variant == "i8"
+    empty_q = sa3.empty_quantized_i8 if i8 else sa3.empty_quantized
+    quantize = sa3.quantize_qkv_i8 if i8 else sa3.quantize_qkv
+    attend = sa3.attn_fwd_i8 if i8 else sa3.attn_fwd
+    qz = empty_q(B, H, N, d, dev)
     ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
     out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -187,8 +194,8 @@ def run_sa3(args, rank, world, local):
         torch.sum(clean, dim=0, out=clean_sum)  # refill L2 with clean, unrelated lines
 
     def step():
-        sa3.quantize_qkv(q, k, v, out=qz, workspace=ws)
-        sa3.attn_fwd(qz, causal=causal, out=out)
+        quantize(q, k, v, out=qz, workspace=ws)
+        attend(qz, causal=causal, out=out)
 
     for _ in range(args.warmup):
         step()
@@ -205,9 +212,9 @@ def run_sa3(args, rank, world, local):
         for i in range(args.steps):
             flush_l2(i)
             ev[i][0].record(stream)
-            sa3.quantize_qkv(q, k, v, out=qz, workspace=ws)
+            quantize(q, k, v, out=qz, workspace=ws)
             ev[i][1].record(stream)
-            sa3.attn_fwd(qz, causal=causal, out=out)
+            attend(qz, causal=causal, out=out)
             ev[i][2].record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -228,7 +235,7 @@ def run_sa3(args, rank, world, local):
     sets = []
     for _ in range(2):
         sets.append(dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
-                         qz=sa3.empty_quantized(B, H, N, d, dev), ws=torch.empty_like(ws),
+                         qz=empty_q(B, H, N, d, dev), ws=torch.empty_like(ws),
                          out=torch.empty_like(out),
                          out_h=torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory(),
                          ready=torch.cuda.Event(), done=torch.cuda.Event(), free=torch.cuda.Event()))
@@ -244,8 +251,8 @@ def run_sa3(args, rank, world, local):
                 b["v"].copy_(vp, non_blocking=True)
                 b["ready"].record(up_s)
             stream.wait_event(b["ready"])
-            sa3.quantize_qkv(b["q"], b["k"], b["v"], out=b["qz"], workspace=b["ws"], stream=stream)
-            sa3.attn_fwd(b["qz"], causal=causal, out=b["out"], stream=stream)
+            quantize(b["q"], b["k"], b["v"], out=b["qz"], workspace=b["ws"], stream=stream)
+            attend(b["qz"], causal=causal, out=b["out"], stream=stream)
             b["done"].record(stream)
             down_s.wait_event(b["done"])
             with torch.cuda.stream(down_s):
@@ -283,10 +290,24 @@ def run_sa3(args, rank, world, local):
         return
     pk, src = peaks()
     ops = w.ops
-    fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
     achieved = ops / (t_attn * 1e-3) / 1e12
-    qk_bytes = 3 * (B * H * N * d * 2) + 3 * (B * H * sa3.padded_len(N) * d // 2) \
-        + 3 * (B * H * sa3.padded_len(N) * d // 16)
+    Np = sa3.padded_len(N)
+    if i8:
+        # half the ops at the int8 rate (2x bf16, nominal), half at the fp16 rate
+        peak = pk["bf16_tflops"] * 4.0 / 3.0
+        peak_src = f"{src} bf16 burst {pk['bf16_tflops']} x 4/3 (QK^T at the nominal int8 rate 2x, P V at 1x)"
+        qk_bytes = 3 * (B * H * N * d * 2) + 2 * (B * H * Np * d) + B * H * d * Np * 2 + 2 * (B * H * Np // 128) * 4
+        dtype = "int8 QK^T (fp32 scale per 128-token tile), fp16 P V, fp32 accumulate"
+        kernel, traffic = "attn8_fwd_kernel<%d>" % d, None
+    else:
+        peak = pk["bf16_tflops"] * FP4_PER_BF16
+        peak_src = f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"
+        qk_bytes = 3 * (B * H * N * d * 2) + 3 * (B * H * Np * d // 2) + 3 * (B * H * Np * d // 16)
+        dtype = "fp4-e2m1 (ue4m3 scales, fp32 accumulate)"
+        kernel = "attn_fwd_kernel<%d>" % d
+        traffic = profiled_traffic("bit_quantized_attention_sa3_b200/csrc/attn.cuh",
+                                   "attn_fwd_kernel_d128_noncausal_b2h16n4096d128.md") \
+            if (d, args.workload) == (128, WORKLOAD) else None
     line = {
         "metric": METRIC,
         "value": round(world * ops / (t_step * 1e-3) / 1e12, 2),
@@ -298,21 +319,20 @@ def run_sa3(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp4-e2m1 (ue4m3 scales, fp32 accumulate)",
+        "dtype": dtype,
         "data": "synthetic (seeded, sa3_inputs.py)",
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": causal,
-                   "step": "sa3_quantize_qkv + sa3_attn_fwd", "l2": "flushed before each step: 256 MiB write, then 256 MiB read of another buffer",
+                   "variant": args.variant,
+                   "step": ("sa3_quantize_qkv_i8 + sa3_attn_fwd_i8" if i8 else "sa3_quantize_qkv + sa3_attn_fwd"),
+                   "l2": "flushed before each step: 256 MiB write, then 256 MiB read of another buffer",
                    "parallelism": f"{world} independent replicas (one batch per GPU)"},
         "attn_only": {"value": round(achieved, 2), "unit": UNIT, "ms": round(t_attn, 4),
                       "frac_of_datasheet_fp4_9000": round(achieved / FP4_DATASHEET_TOPS, 4)},
         "quantize": {"ms": round(t_quant, 4), "GB_per_s": round(qk_bytes / (t_quant * 1e-3) / 1e9, 1),
                      "algorithmic_bytes": qk_bytes},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
-                     "traffic": profiled_traffic("bit_quantized_attention_sa3_b200/csrc/attn.cuh",
-                                                 "attn_fwd_kernel_d128_noncausal_b2h16n4096d128.md"),
-                     "kernel": "attn_fwd_kernel<128>",
-                     "peak_source": f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": kernel, "peak_source": peak_src},
         "e2e": {"value": round(world * ops / (t_e2e * 1e-3) / 1e12, 2), "unit": UNIT, "ms": round(t_e2e, 4),
                 "pipelined": "2 buffer sets; upload, kernels and download on three streams",
                 "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 2},
@@ -320,11 +340,11 @@ def run_sa3(args, rank, world, local):
         "clocks": clk.summary(),
     }
     if world == 1 and not args.skip_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0)
+        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8)
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None):
+def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False):
     """The oracle, as it stands, on the host cores: full quantization plus
     attention for a seeded sample of Q blocks; the full-job time is
     extrapolated from the sampled blocks (non-causal: every block costs
@@ -333,7 +353,7 @@ def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None):
     import oracle
     oracle.build()
     t0 = time.perf_counter()
-    qz = oracle.quantize_qkv(q, k, v)
+    qz = (oracle.quantize_qkv_i8 if i8 else oracle.quantize_qkv)(q, k, v)
     t_quant = time.perf_counter() - t0
     nqb = (w.N + 127) // 128
     total_units = w.B * w.H * nqb
@@ -346,7 +366,7 @@ def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None):
             break
         units = [(int(u) // nqb, int(u) % nqb) for u in chunk]
         t0 = time.perf_counter()
-        oracle.attn_fwd(qz, w.N, w.causal, units=units)
+        (oracle.attn_fwd_i8 if i8 else oracle.attn_fwd)(qz, w.N, w.causal, units=units)
         t_attn += time.perf_counter() - t0
         done += len(chunk)
         if t_quant + t_attn > budget_s or (units_cap and done >= units_cap):

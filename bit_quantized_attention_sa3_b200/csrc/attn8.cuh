@@ -333,15 +333,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 64; ++e)
                     if (e >= lim) s[e >> 5][e & 31] = __float_as_uint(-INFINITY);
             }
-            // partial row maximum: four independent 3-input chains, then combined
-            float mx[4] = {x(0), x(1), x(2), x(3)};
+            // partial row maximum: four 3-input chains over 16 scores each
+            float mx[4];
 #pragma unroll
-            for (int e = 4; e < 64; e += 8) {
-                mx[0] = max3f(mx[0], x(e), x(e + 1));
-                mx[1] = max3f(mx[1], x(e + 2), x(e + 3));
-                mx[2] = max3f(mx[2], x(e + 4), x(e + 5));
-                mx[3] = max3f(mx[3], x(e + 6), x(e + 7));
+            for (int k = 0; k < 4; ++k) mx[k] = x(16 * k);
+#pragma unroll
+            for (int e = 1; e < 15; e += 2) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mx[k] = max3f(mx[k], x(16 * k + e), x(16 * k + e + 1));
             }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], x(16 * k + 15));
             float *xs = xch + (((j & 1) * 2 + i) * 2) * kBlk;
             xs[h * kBlk + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             mbar_arrive(xbar);

@@ -145,3 +145,23 @@ def test_attn_tail_wave_single_tile_units(causal):
     err, cos_gpu, cos_oracle = _run("tiny_b1h2n256d64", {"H": 151, "N": 300}, causal)
     assert err <= TOL, f"rel-L2 vs oracle {err:.3e}"
     assert cos_gpu >= cos_oracle - 1e-3
+
+
+@pytest.mark.gpu
+def test_causal_row0_matches_oracle_exactly():
+    """Row 0 sees key 0 only (P = [1, 0, ...], one code and scale decision):
+    the GPU must give the oracle's bf16(1.03125 * v^_0) to within one bf16
+    ulp, on inputs whose row-0 logits reach far below zero.  (The GPU folds
+    log2(1/s) into the exp2 argument, -m' + log2(1/s) rounded at the size of
+    m', so with logits in the thousands P carries ~1e-4 relative error and
+    some outputs land one ulp away.)"""
+    q, k, v = sa3_inputs.make_qkv("prefill_b4h32n8192d128_causal", shape_override={"B": 1, "H": 32, "N": 1024})
+    B, H, N, d = q.shape
+    qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
+    out = sa3.attn_fwd(qz, causal=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    ref = oracle.attn_fwd(_canonical(qz, B, H, N, d), N, True, units=[(bh, 0) for bh in range(B * H)])
+    got = out[:, :, 0].float().cpu().numpy()
+    want = bits_to_f32(ref[:, :, 0])
+    assert np.all(np.abs(got - want) <= 2.0 ** -7 * np.abs(want))

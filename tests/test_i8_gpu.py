@@ -26,6 +26,7 @@ CASES = [
     ("noncausal_b2h16n4096d128", 77, 1000, {"B": 1, "H": 2}),
     ("noncausal_b2h16n4096d128", 1000, 130, {"B": 1, "H": 2}),
     ("videodit_b1h30n17776d64", 1000, 1000, {"H": 2}),
+    ("prefill_b4h32n8192d128_causal", 2048, 2048, {"B": 1, "H": 4}),
 ]
 
 
@@ -86,3 +87,17 @@ def test_attn_i8_matches_oracle(case, causal):
     err = rel_l2(g, r)
     assert err <= TOL, f"rel-L2 vs oracle {err:.3e}"
     assert cosine(g, e) >= cosine(r, e) - 1e-3
+
+
+@pytest.mark.gpu
+def test_causal_row0_returns_its_value_i8():
+    """Row 0 sees key 0 only, so P = 1 there and the output is V's row 0,
+    whatever its logit: on the prefill workload (outlier channels) some
+    heads' row-0 logit is far below zero, which a wrong running maximum
+    turns into P = 0, l = 0 and NaN."""
+    q, k, v = sa3_inputs.make_qkv("prefill_b4h32n8192d128_causal", shape_override={"B": 1, "H": 32, "N": 1024})
+    qz = sa3.quantize_qkv_i8(q.cuda(), k.cuda(), v.cuda())
+    out = sa3.attn_fwd_i8(qz, causal=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    assert torch.equal(out[:, :, 0].cpu(), v[:, :, 0])
