@@ -14,7 +14,8 @@ Functions follow the method's steps in order:
   attn_fwd         tiled online-softmax attention on the quantized operands
   attn_exact       fp64 softmax attention on the bf16 inputs (no quantization)
   quantize_qkv_i8,
-  attn_fwd_i8      the 8-bit variant: INT8 Q, K per 128-token block, FP16 P, V
+  attn_fwd_i8      the 8-bit variant: INT8 Q, K per 128-token block, FP16 P, V;
+                   optionally the per-row log-sum-exp of the training forward
 Layouts are the canonical ones documented in ``sa3_oracle.c``.
 """
 from __future__ import annotations
@@ -84,7 +85,7 @@ def _load():
         lib.oracle_quantize_qkv_i8.restype = None
         lib.oracle_quantize_qkv_i8.argtypes = [P, P, P, I, I, I, I, I] + [P] * 6
         lib.oracle_attn_fwd_i8.restype = None
-        lib.oracle_attn_fwd_i8.argtypes = [P] * 5 + [I, I, I, I, I, I, F, P, I, P]
+        lib.oracle_attn_fwd_i8.argtypes = [P] * 5 + [I, I, I, I, I, I, F, P, I, P, P]
         lib.oracle_num_threads.restype = I
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -253,20 +254,23 @@ def quantize_qkv_i8(q, k, v) -> dict:
 
 
 def attn_fwd_i8(qz: dict, N: int, causal: bool, sm_scale: float | None = None, units=None,
-                n_kv: int | None = None) -> np.ndarray:
+                n_kv: int | None = None, return_lse: bool = False):
     """8-bit variant attention (readings I3-I5) on quantize_qkv_i8 operands;
-    N query rows, n_kv keys (default qz["n_kv"] or N); bf16 bits [B,H,N,d]."""
+    N query rows, n_kv keys (default qz["n_kv"] or N); bf16 bits [B,H,N,d].
+    With return_lse, also the per-row log-sum-exp of the training forward
+    (reading I6): (out, lse) with lse float32 [B,H,N]."""
     if n_kv is None:
         n_kv = qz.get("n_kv", N)
     B, H, _, d = qz["q_i8"].shape
     if sm_scale is None:
         sm_scale = 1.0 / float(np.sqrt(d))
     out = np.zeros((B, H, N, d), np.uint16)
+    lse = np.full((B, H, N), np.nan, np.float32) if return_lse else None
     u, nu = _units_arr(units)
     arrs = [np.ascontiguousarray(qz[n]) for n in ("q_i8", "q_scale", "k_i8", "k_scale", "vt_f16")]
     _load().oracle_attn_fwd_i8(*[_ptr(a) for a in arrs], B, H, N, n_kv, d, int(bool(causal)), float(sm_scale),
-                               _ptr(u), nu, _ptr(out))
-    return out
+                               _ptr(u), nu, _ptr(out), _ptr(lse))
+    return (out, lse) if return_lse else out
 
 
 def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:

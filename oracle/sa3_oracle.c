@@ -488,6 +488,14 @@ void oracle_attn_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  *     P V; the row sum l accumulates the fp32 P;
  *  I5 O accumulates in fp32 (the summary's ablation finds an FP16
  *     accumulator changes nothing; fp32 is the tensor core's native one).
+ *  I6 the forward used for training ("SageAttention3: Microscaling FP4
+ *     Attention for Inference and An Exploration of 8-Bit Training",
+ *     abstract: 8-bit attention in the forward and backward passes) also
+ *     returns, per query row, the natural-log log-sum-exp of the row's
+ *     scaled logits, which a backward pass needs to rebuild P:
+ *     lse = ln 2 * (m + log2 l), evaluated in fp64 from the final fp32
+ *     running max m (base-2 units) and row sum l; +inf for a row that sees
+ *     no key, so that exp(s - lse) is 0 there.
  * Masks, lengths and the empty-row rule are those of R9, R11, R12. */
 
 /* fp32 -> fp16 bits, round to nearest even, overflow to inf. */
@@ -583,7 +591,7 @@ void oracle_quantize_qkv_i8(const uint16_t *q, const uint16_t *k, const uint16_t
 
 void oracle_attn_fwd_i8(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8, const float *k_scale,
                         const uint16_t *vt_f16, int B, int H, int Nq, int Nkv, int d, int causal,
-                        float sm_scale, const int32_t *units, int n_units, uint16_t *out)
+                        float sm_scale, const int32_t *units, int n_units, uint16_t *out, float *lse)
 {
     const long BH = (long)B * H;
     const int Npq = oracle_padded_len(Nq), Np = oracle_padded_len(Nkv);
@@ -647,6 +655,9 @@ void oracle_attn_fwd_i8(const int8_t *q_i8, const float *q_scale, const int8_t *
             }
             for (int c = 0; c < d; ++c)
                 out[(bh * Nq + row) * d + c] = l > 0.0f ? oracle_f32_to_bf16(O[c] / l) : 0;
+            if (lse)  /* I6 */
+                lse[bh * Nq + row] = l > 0.0f ? (float)(0.69314718055994531 * ((double)m + log2((double)l)))
+                                              : INFINITY;
         }
         free(O);
         free(vhat);

@@ -117,3 +117,70 @@ def test_int8_variant_is_more_accurate_than_fp4():
     fp4 = oracle.bf16_bits_to_f32(oracle.attn_fwd(oracle.quantize_qkv(q, k, v), 256, False)).astype(np.float64).ravel()
     cos = lambda a, b: a @ b / np.sqrt((a @ a) * (b @ b))
     assert cos(i8, ex) >= 0.999 and cos(i8, ex) > cos(fp4, ex)
+
+
+# ---- log-sum-exp of the training forward (reading I6)
+
+@pytest.mark.parametrize("Nq,Nkv,causal", [(300, 300, False), (300, 300, True), (70, 300, True),
+                                           (300, 70, True), (70, 300, False)])
+def test_lse_with_zero_scale_is_log_of_visible_count(Nq, Nkv, causal):
+    """sm_scale = 0 makes every visible logit 0, so P = 1 on each visible
+    key and lse = ln(number of keys the row sees); a row that sees none
+    gets +inf."""
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": max(Nq, Nkv)})
+    q, k, v = q[:, :, :Nq].contiguous(), k[:, :, :Nkv].contiguous(), v[:, :, :Nkv].contiguous()
+    _, lse = oracle.attn_fwd_i8(oracle.quantize_qkv_i8(q, k, v), Nq, causal, sm_scale=0.0, return_lse=True)
+    rows = np.arange(Nq)
+    count = np.minimum(rows + 1 + (Nkv - Nq), Nkv) if causal else np.full(Nq, Nkv)
+    want = np.where(count > 0, np.log(np.maximum(count, 1)), np.inf).astype(np.float32)
+    assert np.array_equal(np.isinf(lse[0, 0]), count <= 0)
+    np.testing.assert_allclose(lse[..., count > 0], np.broadcast_to(want[count > 0], lse[..., count > 0].shape),
+                               rtol=2e-7, atol=0)
+
+
+@pytest.mark.parametrize("Nq,Nkv,causal", [(300, 300, False), (300, 300, True), (70, 300, True), (300, 70, True)])
+def test_lse_agrees_with_bruteforce_logsumexp(Nq, Nkv, causal):
+    """fp64 logsumexp of sm_scale * (Q^ K^T) on the dequantized INT8
+    operands.  The oracle's t is fp32 (a few roundings of a product whose
+    magnitude stays below 64 here) and l an fp32 sum, so 1e-5 absolute."""
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": max(Nq, Nkv)})
+    q, k, v = q[:, :, :Nq].contiguous(), k[:, :, :Nkv].contiguous(), v[:, :, :Nkv].contiguous()
+    d = q.shape[-1]
+    qz = oracle.quantize_qkv_i8(q, k, v)
+    _, lse = oracle.attn_fwd_i8(qz, Nq, causal, return_lse=True)
+    qh, kh, _ = _dequant(qz)
+    s = qh[:, :, :Nq] @ np.swapaxes(kh[:, :, :Nkv], -1, -2) / np.sqrt(d)
+    assert np.abs(s).max() < 64
+    if causal:
+        vis = np.arange(Nkv)[None, :] <= np.arange(Nq)[:, None] + (Nkv - Nq)
+        s = np.where(vis, s, -np.inf)
+    with np.errstate(divide="ignore"):
+        mx = s.max(-1, keepdims=True)
+        ref = (mx + np.log(np.exp(s - np.where(np.isfinite(mx), mx, 0)).sum(-1, keepdims=True)))[..., 0]
+    live = np.isfinite(ref)
+    assert np.array_equal(np.isinf(lse), ~live) and (lse[~live] > 0).all()
+    assert np.abs(lse[live] - ref[live]).max() <= 1e-5
+
+
+def test_lse_reconstructs_the_output():
+    """What a backward pass does with lse: P = exp(s - lse) has rows that sum
+    to 1 and P V^ gives the forward's output (to the FP16 rounding of P)."""
+    N, d = 260, 64
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": N})
+    qz = oracle.quantize_qkv_i8(q, k, v)
+    out, lse = oracle.attn_fwd_i8(qz, N, True, return_lse=True)
+    qh, kh, vh = _dequant(qz)
+    s = qh[:, :, :N] @ np.swapaxes(kh[:, :, :N], -1, -2) / np.sqrt(d) + np.triu(np.full((N, N), -np.inf), 1)
+    pr = np.exp(s - lse[..., None].astype(np.float64))
+    np.testing.assert_allclose(pr.sum(-1), 1.0, rtol=0, atol=2e-5)
+    o = oracle.bf16_bits_to_f32(out).astype(np.float64)
+    ref = pr @ vh[:, :, :N]
+    assert np.linalg.norm(o - ref) / np.linalg.norm(ref) <= 2e-3
+
+
+def test_lse_is_optional_and_leaves_the_output_unchanged():
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64")
+    qz = oracle.quantize_qkv_i8(q, k, v)
+    a = oracle.attn_fwd_i8(qz, 256, True)
+    b, _ = oracle.attn_fwd_i8(qz, 256, True, return_lse=True)
+    assert np.array_equal(a, b)
