@@ -55,9 +55,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sa3", choices=["sa3", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=list(sa3_inputs.WORKLOADS))
-    ap.add_argument("--variant", default="fp4", choices=["fp4", "i8"],
+    ap.add_argument("--variant", default="fp4", choices=["fp4", "i8", "i8_train"],
                     help="fp4: the microscaled FP4 path (the headline); i8: the 8-bit variant "
-                         "(INT8 QK^T, FP16 P V)")
+                         "(INT8 QK^T, FP16 P V); i8_train: the 8-bit forward used for training "
+                         "(also writes the per-row log-sum-exp)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
     return ap.parse_args()
@@ -177,10 +178,16 @@ def run_sa3(args, rank, world, local):
     B, H, N, d, causal = w.B, w.H, w.N, w.d, w.causal
     q_h, k_h, v_h = sa3_inputs.make_qkv(w, seed=rank)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    i8 = args.variant == "i8"
+    i8 = args.variant in ("i8", "i8_train")
+    train = args.variant == "i8_train"
     empty_q = sa3.empty_quantized_i8 if i8 else sa3.empty_quantized
     quantize = sa3.quantize_qkv_i8 if i8 else sa3.quantize_qkv
-    attend = sa3.attn_fwd_i8 if i8 else sa3.attn_fwd
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if train else None
+
+    def attend(qz, causal, out, stream=None, lse=lse):
+        if i8:
+            return sa3.attn_fwd_i8(qz, causal=causal, out=out, stream=stream, lse=lse)
+        return sa3.attn_fwd(qz, causal=causal, out=out, stream=stream)
     qz = empty_q(B, H, N, d, dev)
     ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
     out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
@@ -238,6 +245,8 @@ def run_sa3(args, rank, world, local):
                          qz=empty_q(B, H, N, d, dev), ws=torch.empty_like(ws),
                          out=torch.empty_like(out),
                          out_h=torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory(),
+                         lse=torch.empty_like(lse) if train else None,
+                         lse_h=torch.empty((B, H, N), dtype=torch.float32).pin_memory() if train else None,
                          ready=torch.cuda.Event(), done=torch.cuda.Event(), free=torch.cuda.Event()))
 
     def e2e_run(n):
@@ -252,11 +261,13 @@ def run_sa3(args, rank, world, local):
                 b["ready"].record(up_s)
             stream.wait_event(b["ready"])
             quantize(b["q"], b["k"], b["v"], out=b["qz"], workspace=b["ws"], stream=stream)
-            attend(b["qz"], causal=causal, out=b["out"], stream=stream)
+            attend(b["qz"], causal=causal, out=b["out"], stream=stream, lse=b["lse"])
             b["done"].record(stream)
             down_s.wait_event(b["done"])
             with torch.cuda.stream(down_s):
                 b["out_h"].copy_(b["out"], non_blocking=True)
+                if train:
+                    b["lse_h"].copy_(b["lse"], non_blocking=True)
                 b["free"].record(down_s)
         stream.wait_stream(up_s)
         stream.wait_stream(down_s)
@@ -274,6 +285,8 @@ def run_sa3(args, rank, world, local):
     e2e_ms = e0.elapsed_time(e1) / n_e2e
     if not torch.equal(sets[(n_e2e - 1) % 2]["out_h"], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
+    if train and not torch.equal(sets[(n_e2e - 1) % 2]["lse_h"], lse.cpu()):
+        raise RuntimeError("end-to-end log-sum-exp differs from the device-resident run")
 
     def gmax(x):
         if world == 1:
@@ -323,7 +336,8 @@ def run_sa3(args, rank, world, local):
         "data": "synthetic (seeded, sa3_inputs.py)",
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": causal,
                    "variant": args.variant,
-                   "step": ("sa3_quantize_qkv_i8 + sa3_attn_fwd_i8" if i8 else "sa3_quantize_qkv + sa3_attn_fwd"),
+                   "step": ("sa3_quantize_qkv_i8 + sa3_attn_fwd_i8_lse" if train else
+                            "sa3_quantize_qkv_i8 + sa3_attn_fwd_i8" if i8 else "sa3_quantize_qkv + sa3_attn_fwd"),
                    "l2": "flushed before each step: 256 MiB write, then 256 MiB read of another buffer",
                    "parallelism": f"{world} independent replicas (one batch per GPU)"},
         "attn_only": {"value": round(achieved, 2), "unit": UNIT, "ms": round(t_attn, 4),
@@ -335,16 +349,17 @@ def run_sa3(args, rank, world, local):
                      "kernel": kernel, "peak_source": peak_src},
         "e2e": {"value": round(world * ops / (t_e2e * 1e-3) / 1e12, 2), "unit": UNIT, "ms": round(t_e2e, 4),
                 "pipelined": "2 buffer sets; upload, kernels and download on three streams",
-                "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 2},
+                "h2d_bytes_per_step": 3 * B * H * N * d * 2,
+                "d2h_bytes_per_step": B * H * N * d * 2 + (B * H * N * 4 if train else 0)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.skip_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8)
+        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8, train=train)
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False):
+def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=False):
     """The oracle, as it stands, on the host cores: full quantization plus
     attention for a seeded sample of Q blocks; the full-job time is
     extrapolated from the sampled blocks (non-causal: every block costs
@@ -366,7 +381,10 @@ def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False):
             break
         units = [(int(u) // nqb, int(u) % nqb) for u in chunk]
         t0 = time.perf_counter()
-        (oracle.attn_fwd_i8 if i8 else oracle.attn_fwd)(qz, w.N, w.causal, units=units)
+        if i8:
+            oracle.attn_fwd_i8(qz, w.N, w.causal, units=units, return_lse=train)
+        else:
+            oracle.attn_fwd(qz, w.N, w.causal, units=units)
         t_attn += time.perf_counter() - t0
         done += len(chunk)
         if t_quant + t_attn > budget_s or (units_cap and done >= units_cap):
@@ -392,8 +410,9 @@ def run_reference(args, rank, world):
     q, k, v = sa3_inputs.make_qkv(w, seed=0)
     per_step = []
     budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
+    i8, train = args.variant in ("i8", "i8_train"), args.variant == "i8_train"
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, q, k, v, budget_s=budget)
+        cb = cpu_baseline(w, q, k, v, budget_s=budget, i8=i8, train=train)
         if i >= args.warmup:
             per_step.append(cb)
     vals = [c["value"] for c in per_step]
@@ -405,6 +424,7 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)",
         "data": "synthetic (seeded, sa3_inputs.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "variant": args.variant,
                    "step": "oracle quantize + tiled attention (sampled, extrapolated)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"]},

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
             L.sa3_quantize_qkv_i8.argtypes = [P, P, P, I, I, I, I, I, ctypes.POINTER(_QKVI8), P, ctypes.c_size_t, P]
             L.sa3_attn_fwd_i8.restype = I
             L.sa3_attn_fwd_i8.argtypes = [ctypes.POINTER(_QKVI8), I, I, I, I, I, I, F, P, P]
+            L.sa3_attn_fwd_i8_lse.restype = I
+            L.sa3_attn_fwd_i8_lse.argtypes = [ctypes.POINTER(_QKVI8), I, I, I, I, I, I, F, P, P, P]
             L.sa3_device_status.restype = I
             L.sa3_device_status.argtypes = [P]
             _lib = L
@@ -268,19 +270,33 @@ def quantize_qkv_i8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Quan
 
 
 def attn_fwd_i8(qz: QuantizedQKVI8, causal: bool = False, sm_scale: float | None = None,
-                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """sa3_attn_fwd_i8: 8-bit attention (INT8 QK^T, FP16 P V); bf16 [B,H,Nq,d]."""
+                out: torch.Tensor | None = None, stream=None, lse: torch.Tensor | bool | None = None):
+    """sa3_attn_fwd_i8: 8-bit attention (INT8 QK^T, FP16 P V); bf16 [B,H,Nq,d].
+
+    With ``lse`` (True, or a float32 [B,H,Nq] tensor to fill) this is the
+    training forward, sa3_attn_fwd_i8_lse: it also writes each row's
+    log-sum-exp and returns ``(out, lse)``."""
     B, H, N, d, Nq = qz.B, qz.H, qz.N, qz.d, qz.Nq
     if out is None:
         out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=qz.q_i8.device)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
+    if lse is True:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=qz.q_i8.device)
     st = qz.struct()
-    rc = lib().sa3_attn_fwd_i8(ctypes.byref(st), B, H, Nq, N, d, int(bool(causal)), float(sm_scale),
-                               out.data_ptr(), _stream_ptr(stream))
+    if lse is None or lse is False:
+        rc = lib().sa3_attn_fwd_i8(ctypes.byref(st), B, H, Nq, N, d, int(bool(causal)), float(sm_scale),
+                                   out.data_ptr(), _stream_ptr(stream))
+        if rc != SA3_OK:
+            raise Sa3Error(rc, "sa3_attn_fwd_i8")
+        return out
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.numel() != B * H * Nq:
+        raise ValueError("lse must be a contiguous float32 tensor of B*H*Nq elements")
+    rc = lib().sa3_attn_fwd_i8_lse(ctypes.byref(st), B, H, Nq, N, d, int(bool(causal)), float(sm_scale),
+                                   out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
     if rc != SA3_OK:
-        raise Sa3Error(rc, "sa3_attn_fwd_i8")
-    return out
+        raise Sa3Error(rc, "sa3_attn_fwd_i8_lse")
+    return out, lse
 
 
 def device_status(stream=None) -> int:

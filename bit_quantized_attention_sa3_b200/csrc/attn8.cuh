@@ -9,7 +9,8 @@
 //   m' = max(m, rowmax t), alpha = 2^(m - m'), P = 2^(t - m'),
 //   l = alpha l + rowsum P, P16 = fp16(P)
 //   O = alpha O + P16 V16_j             tcgen05.mma kind::f16, fp32 in TMEM
-// and out = bf16(O / l).
+// and out = bf16(O / l); optionally lse = ln 2 (m + log2 l) per row, the
+// softmax statistic that a backward pass of the training forward reuses.
 //
 // Same CTA organisation as the FP4 kernel (attn.cuh): two Q tiles per CTA,
 // 16 softmax warps (two threads per row, exchanging partial row maxima),
@@ -422,6 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(xbar);
             ok = warp_wait(xbar, n_i & 1, abort_flag);
             l_row = xl[r] + xl[kBlk + r];
+            // log-sum-exp of the row's scaled logits (natural log) for a
+            // backward pass: ln 2 (m + log2 l); +inf where no key was seen
+            if (ok && p.lse && h == 0 && grow < p.Nq)
+                p.lse[static_cast<size_t>(bh) * p.Nq + grow] =
+                    l_row > 0.0f ? (m + log2f(l_row)) * 0.693147182f : INFINITY;
         }
         if (ok && n_i > 0 && warp_wait(bars + kBarPvDone + i, (n_i - 1) & 1, abort_flag)) {
             tc_fence_after();
@@ -450,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.Nq + grow) * D + h * (D / 2));
 #pragma unroll
             for (int v = 0; v < D / 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            if (p.lse && h == 0) p.lse[static_cast<size_t>(bh) * p.Nq + grow] = INFINITY;
         }
     }
 

@@ -257,14 +257,15 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
                : SA3_ERR_CUDA;
 }
 
-int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
-                    void *out, struct CUstream_st *stream) {
+int sa3_attn_fwd_i8_lse(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                        void *out, float *lse, struct CUstream_st *stream) {
     int rc = check_shape(B, H, Nq, d);
     if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
     if (!in || !in->q_i8 || !in->q_scale || !in->k_i8 || !in->k_scale || !in->vt_f16 || !aligned16(in->q_i8) ||
         !aligned16(in->k_i8) || !aligned16(in->vt_f16))
         return SA3_ERR_INVALID_ARG;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SA3_ERR_INVALID_ARG;
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
     const int BH = B * H;
@@ -281,6 +282,7 @@ int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, 
     p.q_scale = in->q_scale;
     p.k_scale = in->k_scale;
     p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
     p.BH = BH;
     p.N = Nkv;
     p.Np = Np;
@@ -291,6 +293,11 @@ int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, 
     return sa3::launch_attn_i8(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA3_OK
                : SA3_ERR_CUDA;
+}
+
+int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                    void *out, struct CUstream_st *stream) {
+    return sa3_attn_fwd_i8_lse(in, B, H, Nq, Nkv, d, causal, sm_scale, out, nullptr, stream);
 }
 
 int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,

@@ -37,6 +37,7 @@ struct AttnParams {
     const float *q_scale;  // 8-bit variant: fp32 scale per 128-token tile of Q
     const float *k_scale;  // ... and of K
     __nv_bfloat16 *out;
+    float *lse;        // 8-bit variant: per-row log-sum-exp (natural log), or null
     int BH;
     int N;             // key / value tokens
     int Np;            // N rounded up to 128

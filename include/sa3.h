@@ -238,6 +238,28 @@ int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d,
                     struct CUstream_st *stream);
 
 /*
+ * sa3_attn_fwd_i8_lse -- the 8-bit forward as used for training
+ * ("SageAttention3: Microscaling FP4 Attention for Inference and An
+ * Exploration of 8-Bit Training", abstract: 8-bit attention in both the
+ * forward and the backward pass).  The backward pass needs each row's
+ * softmax normaliser to rebuild P; this call is sa3_attn_fwd_i8 that also
+ * writes it:
+ *
+ *   lse : fp32 [B][H][Nq], device, 4-byte aligned, caller-owned.
+ *         lse[r] = ln 2 * (m + log2 l), m the row's final running maximum
+ *         of t (base-2 units, t as above) and l its fp32 row sum of P, so
+ *         lse = ln sum_j exp(sm_scale * s_q s_k * S_rj) over the keys the
+ *         row sees, up to fp32 rounding.  A row that sees no key gets +inf
+ *         (its P = exp(s - lse) is then 0).
+ *
+ * lse == NULL is sa3_attn_fwd_i8.  A misaligned lse: SA3_ERR_INVALID_ARG.
+ * Other arguments, errors and asynchrony as in sa3_attn_fwd_i8.
+ */
+int sa3_attn_fwd_i8_lse(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d,
+                        int causal, float sm_scale, void *out, float *lse,
+                        struct CUstream_st *stream);
+
+/*
  * sa3_quantize_qkv_noalloc -- sa3_quantize_qkv without a caller workspace.
  *
  * There is no counterpart in the paper: this is a convenience for callers

@@ -26,7 +26,7 @@ def lib():
 
 
 def test_header_declares_the_boundary():
-    assert _declared() == ["sa3_attn_fwd", "sa3_attn_fwd_i8", "sa3_attn_fwd_lens", "sa3_device_status",
+    assert _declared() == ["sa3_attn_fwd", "sa3_attn_fwd_i8", "sa3_attn_fwd_i8_lse", "sa3_attn_fwd_lens", "sa3_device_status",
                            "sa3_quantize_qkv", "sa3_quantize_qkv_i8", "sa3_quantize_qkv_lens",
                            "sa3_quantize_qkv_noalloc", "sa3_selftest_wait_timeout", "sa3_version"]
 
