@@ -59,9 +59,19 @@ def parse():
                     help="fp4: the microscaled FP4 path (the headline); i8: the 8-bit variant "
                          "(INT8 QK^T, FP16 P V); i8_train: the 8-bit forward used for training "
                          "(also writes the per-row log-sum-exp)")
+    ap.add_argument("--nq", type=int, default=0,
+                    help="query tokens (default: the workload's N); keys and values keep N "
+                         "(sa3_*_lens; causal aligns the last query with the last key)")
+    ap.add_argument("--p-two-level", action="store_true",
+                    help="fp4 only: P pre-scaled by 2^11 before it is microscaled (SA3_P_TWO_LEVEL)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.p_two_level and args.variant != "fp4":
+        ap.error("--p-two-level applies to the fp4 variant only")
+    if args.nq < 0:
+        ap.error("--nq must be positive")
+    return args
 
 
 def dist_init(n):
@@ -170,27 +180,51 @@ def profiled_traffic(kernel_src: str, profile: str):
     return None
 
 
+def attn_ops(w, Nq):
+    """4*d per visible (query, key) pair: the workload's own count (4*B*H*N^2*d,
+    halved for causal) when Nq == N, else the exact count of pairs that the
+    mask leaves (causal: query r sees keys 0 .. r + N - Nq)."""
+    if Nq == w.N:
+        return w.ops
+    if not w.causal:
+        return 4.0 * w.B * w.H * Nq * w.N * w.d
+    off = w.N - Nq
+    pairs = sum(min(max(r + off + 1, 0), w.N) for r in range(Nq))
+    return 4.0 * w.B * w.H * pairs * w.d
+
+
+def make_inputs(w, Nq, seed):
+    """The workload's seeded q, k, v; q cut to (or drawn with) Nq tokens."""
+    if Nq <= w.N:
+        q, k, v = sa3_inputs.make_qkv(w, seed=seed)
+        return (q[:, :, :Nq].contiguous() if Nq < w.N else q), k, v
+    q, k, v = sa3_inputs.make_qkv(w, seed=seed, shape_override={"N": Nq})
+    return q, k[:, :, :w.N].contiguous(), v[:, :, :w.N].contiguous()
+
+
 def run_sa3(args, rank, world, local):
     import bit_quantized_attention_sa3_b200 as sa3
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = sa3_inputs.WORKLOADS[args.workload]
     B, H, N, d, causal = w.B, w.H, w.N, w.d, w.causal
-    q_h, k_h, v_h = sa3_inputs.make_qkv(w, seed=rank)
+    Nq = args.nq or N
+    two = bool(args.p_two_level)
+    q_h, k_h, v_h = make_inputs(w, Nq, seed=rank)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     i8 = args.variant in ("i8", "i8_train")
     train = args.variant == "i8_train"
     empty_q = sa3.empty_quantized_i8 if i8 else sa3.empty_quantized
     quantize = sa3.quantize_qkv_i8 if i8 else sa3.quantize_qkv
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if train else None
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev) if train else None
 
     def attend(qz, causal, out, stream=None, lse=lse):
         if i8:
             return sa3.attn_fwd_i8(qz, causal=causal, out=out, stream=stream, lse=lse)
-        return sa3.attn_fwd(qz, causal=causal, out=out, stream=stream)
-    qz = empty_q(B, H, N, d, dev)
+        return sa3.attn_fwd(qz, causal=causal, out=out, stream=stream, p_two_level=two)
+    qz = empty_q(B, H, N, d, dev, Nq=Nq)
     ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
-    out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     clean_sum = torch.empty((), dtype=torch.float32, device=dev)
@@ -242,11 +276,11 @@ def run_sa3(args, rank, world, local):
     sets = []
     for _ in range(2):
         sets.append(dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
-                         qz=empty_q(B, H, N, d, dev), ws=torch.empty_like(ws),
+                         qz=empty_q(B, H, N, d, dev, Nq=Nq), ws=torch.empty_like(ws),
                          out=torch.empty_like(out),
-                         out_h=torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory(),
+                         out_h=torch.empty((B, H, Nq, d), dtype=torch.bfloat16).pin_memory(),
                          lse=torch.empty_like(lse) if train else None,
-                         lse_h=torch.empty((B, H, N), dtype=torch.float32).pin_memory() if train else None,
+                         lse_h=torch.empty((B, H, Nq), dtype=torch.float32).pin_memory() if train else None,
                          ready=torch.cuda.Event(), done=torch.cuda.Event(), free=torch.cuda.Event()))
 
     def e2e_run(n):
@@ -302,25 +336,26 @@ def run_sa3(args, rank, world, local):
     if rank != 0:
         return
     pk, src = peaks()
-    ops = w.ops
+    ops = attn_ops(w, Nq)
     achieved = ops / (t_attn * 1e-3) / 1e12
-    Np = sa3.padded_len(N)
+    Np, Npq = sa3.padded_len(N), sa3.padded_len(Nq)
+    rd = B * H * d * 2 * (Nq + 2 * N)           # bf16 q, k, v read once
     if i8:
         # half the ops at the int8 rate (2x bf16, nominal), half at the fp16 rate
         peak = pk["bf16_tflops"] * 4.0 / 3.0
         peak_src = f"{src} bf16 burst {pk['bf16_tflops']} x 4/3 (QK^T at the nominal int8 rate 2x, P V at 1x)"
-        qk_bytes = 3 * (B * H * N * d * 2) + 2 * (B * H * Np * d) + B * H * d * Np * 2 + 2 * (B * H * Np // 128) * 4
+        qk_bytes = rd + B * H * d * (Npq + Np) + B * H * d * Np * 2 + B * H * ((Npq + Np) // 128) * 4
         dtype = "int8 QK^T (fp32 scale per 128-token tile), fp16 P V, fp32 accumulate"
         kernel, traffic = "attn8_fwd_kernel<%d>" % d, None
     else:
         peak = pk["bf16_tflops"] * FP4_PER_BF16
         peak_src = f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"
-        qk_bytes = 3 * (B * H * N * d * 2) + 3 * (B * H * Np * d // 2) + 3 * (B * H * Np * d // 16)
+        qk_bytes = rd + B * H * d * (Npq + 2 * Np) // 2 + B * H * d * (Npq + 2 * Np) // 16
         dtype = "fp4-e2m1 (ue4m3 scales, fp32 accumulate)"
         kernel = "attn_fwd_kernel<%d>" % d
         traffic = profiled_traffic("bit_quantized_attention_sa3_b200/csrc/attn.cuh",
                                    "attn_fwd_kernel_d128_noncausal_b2h16n4096d128.md") \
-            if (d, args.workload) == (128, WORKLOAD) else None
+            if (d, args.workload, Nq, two) == (128, WORKLOAD, N, False) else None
     line = {
         "metric": METRIC,
         "value": round(world * ops / (t_step * 1e-3) / 1e12, 2),
@@ -349,28 +384,34 @@ def run_sa3(args, rank, world, local):
                      "kernel": kernel, "peak_source": peak_src},
         "e2e": {"value": round(world * ops / (t_e2e * 1e-3) / 1e12, 2), "unit": UNIT, "ms": round(t_e2e, 4),
                 "pipelined": "2 buffer sets; upload, kernels and download on three streams",
-                "h2d_bytes_per_step": 3 * B * H * N * d * 2,
-                "d2h_bytes_per_step": B * H * N * d * 2 + (B * H * N * 4 if train else 0)},
+                "h2d_bytes_per_step": rd,
+                "d2h_bytes_per_step": B * H * Nq * d * 2 + (B * H * Nq * 4 if train else 0)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
+    if Nq != N:
+        line["config"]["Nq"] = Nq
+        line["config"]["ops"] = "4*d per (query, key) pair the mask leaves"
+    if two:
+        line["config"]["p_two_level"] = True
     if world == 1 and not args.skip_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8, train=train)
+        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8, train=train, two=two)
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=False):
+def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=False, two=False):
     """The oracle, as it stands, on the host cores: full quantization plus
     attention for a seeded sample of Q blocks; the full-job time is
-    extrapolated from the sampled blocks (non-causal: every block costs
-    the same)."""
+    extrapolated from the sampled blocks, each weighted by the KV blocks it
+    processes (non-causal: all the same)."""
     import numpy as np
     import oracle
     oracle.build()
+    Nq, N = q.shape[2], k.shape[2]
     t0 = time.perf_counter()
     qz = (oracle.quantize_qkv_i8 if i8 else oracle.quantize_qkv)(q, k, v)
     t_quant = time.perf_counter() - t0
-    nqb = (w.N + 127) // 128
+    nqb, nkv = (Nq + 127) // 128, (N + 127) // 128
     total_units = w.B * w.H * nqb
     rng = np.random.default_rng(0)
     order = rng.permutation(total_units)
@@ -382,21 +423,23 @@ def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=Fals
         units = [(int(u) // nqb, int(u) % nqb) for u in chunk]
         t0 = time.perf_counter()
         if i8:
-            oracle.attn_fwd_i8(qz, w.N, w.causal, units=units, return_lse=train)
+            oracle.attn_fwd_i8(qz, Nq, w.causal, units=units, return_lse=train)
         else:
-            oracle.attn_fwd(qz, w.N, w.causal, units=units)
+            oracle.attn_fwd(qz, Nq, w.causal, units=units, p_two_level=two)
         t_attn += time.perf_counter() - t0
         done += len(chunk)
         if t_quant + t_attn > budget_s or (units_cap and done >= units_cap):
             break
         n = min(4 * n, 256)
     if w.causal:
-        weights = np.array([(u % nqb) + 1 for u in range(total_units)], float)
-        frac = weights[order[:done]].sum() / weights.sum()
+        last = np.arange(nqb) * 128 + 127 + (N - Nq)
+        per_tile = np.clip(np.where(last < 0, 0, last // 128 + 1), 0, nkv).astype(float)
+        weights = per_tile[np.arange(total_units) % nqb]
+        frac = weights[order[:done]].sum() / max(weights.sum(), 1.0)
     else:
         frac = done / total_units
     t_full = t_quant + t_attn / frac
-    return {"value": round(w.ops / t_full / 1e12, 6), "unit": UNIT, "cores": oracle.num_threads(),
+    return {"value": round(attn_ops(w, Nq) / t_full / 1e12, 6), "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": (f"full quantization ({t_quant:.2f} s) + attention for {done} of {total_units} "
                        f"Q blocks ({t_attn:.2f} s), extrapolated to the whole {w.name} job "
@@ -407,12 +450,13 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     w = sa3_inputs.WORKLOADS[args.workload]
-    q, k, v = sa3_inputs.make_qkv(w, seed=0)
+    Nq = args.nq or w.N
+    q, k, v = make_inputs(w, Nq, seed=0)
     per_step = []
     budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
     i8, train = args.variant in ("i8", "i8_train"), args.variant == "i8_train"
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, q, k, v, budget_s=budget, i8=i8, train=train)
+        cb = cpu_baseline(w, q, k, v, budget_s=budget, i8=i8, train=train, two=bool(args.p_two_level))
         if i >= args.warmup:
             per_step.append(cb)
     vals = [c["value"] for c in per_step]
@@ -420,11 +464,12 @@ def run_reference(args, rank, world):
     last = per_step[-1]
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(w.ops / (value * 1e12) * 1e3, 3),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(attn_ops(w, Nq) / (value * 1e12) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)",
         "data": "synthetic (seeded, sa3_inputs.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                   "variant": args.variant,
+                   "variant": args.variant, **({"Nq": Nq} if Nq != w.N else {}),
+                   **({"p_two_level": True} if args.p_two_level else {}),
                    "step": "oracle quantize + tiled attention (sampled, extrapolated)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"]},
