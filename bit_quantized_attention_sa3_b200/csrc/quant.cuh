@@ -113,7 +113,7 @@ __device__ __forceinline__ float amax16(const uint64_t (&x2)[8]) {
 template <int D, bool kSmooth>
 __device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N, int tile,
                                         const float *__restrict__ neg_mean, const float *__restrict__ rcp_lut,
-                                        uint8_t *__restrict__ codes, uint8_t *__restrict__ sf) {
+                                        uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, bool st32) {
     constexpr int kBpt = D / 32;  // 16-element blocks per thread (4 or 2), consecutive along d
     const int row = static_cast<int>(threadIdx.x) >> 1;
     const int part = static_cast<int>(threadIdx.x) & 1;
@@ -146,8 +146,12 @@ __device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N
     }
     uint8_t *dst = codes + static_cast<size_t>(t) * (D / 2) + part * (kBpt * 8);
     if constexpr (kBpt == 4) {
-        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        if (st32) {
+            st_global_v8(dst, cw);
+        } else {
+            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        }
         // blocks 4*part .. 4*part+3 are the four columns of atom `part`
         *reinterpret_cast<uint32_t *>(sf + static_cast<size_t>(tile * 2 + part) * 512 + atom_off(row, 0)) = scw;
     } else {
@@ -224,7 +228,7 @@ __device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int Np
 template <int D, bool kSmooth>
 __device__ __forceinline__ void qk_tile_i8(const uint8_t *__restrict__ stage, int N, int tile,
                                            const float *__restrict__ neg_mean, int8_t *__restrict__ codes,
-                                           float *__restrict__ scale_out, float *red) {
+                                           float *__restrict__ scale_out, float *red, bool st32) {
     constexpr int kCh = D / 2;  // channels per thread
     const int row = static_cast<int>(threadIdx.x) >> 1;
     const int part = static_cast<int>(threadIdx.x) & 1;
@@ -269,11 +273,22 @@ __device__ __forceinline__ void qk_tile_i8(const uint8_t *__restrict__ stage, in
         }
         pk[i] = word;
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(codes + static_cast<size_t>(t) * D + part * kCh);
+    int8_t *dst = codes + static_cast<size_t>(t) * D + part * kCh;
+    if (st32) {
 #pragma unroll
-    for (int i = 0; i < kCh / 16; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int i = 0; i < kCh / 32; ++i) {
+            const uint32_t w[8] = {pk[8 * i], pk[8 * i + 1], pk[8 * i + 2], pk[8 * i + 3],
+                                   pk[8 * i + 4], pk[8 * i + 5], pk[8 * i + 6], pk[8 * i + 7]};
+            st_global_v8(dst + 32 * i, w);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < kCh / 16; ++i)
+            reinterpret_cast<uint4 *>(dst)[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
     if (threadIdx.x == 0) scale_out[tile] = s;
-    __syncthreads();  // red is rewritten by the next tile
+    // red is rewritten by the next Q or K tile only after the caller's
+    // __syncthreads that follows every tile
 }
 
 // One staged 128-token tile of V as FP16 (round to nearest even), stored
@@ -282,7 +297,7 @@ __device__ __forceinline__ void qk_tile_i8(const uint8_t *__restrict__ stage, in
 // channel and block.
 template <int D>
 __device__ __forceinline__ void v_tile_f16(const uint8_t *__restrict__ stage, int Np, int tile,
-                                           uint8_t *__restrict__ vt) {
+                                           uint8_t *__restrict__ vt, bool st32) {
     constexpr int kPairs = D / 2;
     constexpr int kTbpt = D / 64;
     const int cp = static_cast<int>(threadIdx.x) % kPairs;
@@ -303,10 +318,15 @@ __device__ __forceinline__ void v_tile_f16(const uint8_t *__restrict__ stage, in
         }
         uint8_t *r0 = vt + (static_cast<size_t>(2 * cp) * Np + tile * kTile + tb * 16) * 2;
         uint8_t *r1 = r0 + static_cast<size_t>(Np) * 2;
-        reinterpret_cast<uint4 *>(r0)[0] = make_uint4(h0[0], h0[1], h0[2], h0[3]);
-        reinterpret_cast<uint4 *>(r0)[1] = make_uint4(h0[4], h0[5], h0[6], h0[7]);
-        reinterpret_cast<uint4 *>(r1)[0] = make_uint4(h1[0], h1[1], h1[2], h1[3]);
-        reinterpret_cast<uint4 *>(r1)[1] = make_uint4(h1[4], h1[5], h1[6], h1[7]);
+        if (st32) {
+            st_global_v8(r0, h0);
+            st_global_v8(r1, h1);
+        } else {
+            reinterpret_cast<uint4 *>(r0)[0] = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+            reinterpret_cast<uint4 *>(r0)[1] = make_uint4(h0[4], h0[5], h0[6], h0[7]);
+            reinterpret_cast<uint4 *>(r1)[0] = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+            reinterpret_cast<uint4 *>(r1)[1] = make_uint4(h1[4], h1[5], h1[6], h1[7]);
+        }
     }
 }
 
@@ -535,14 +555,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 qk_tile_i8<D, false>(st, p.Nq, t.tile, nullptr,
                                      reinterpret_cast<int8_t *>(p.q_fp4) + static_cast<size_t>(t.bh) * p.Npq * D,
                                      p.q_scale + static_cast<size_t>(t.bh) * (p.Npq / kTile),
-                                     reinterpret_cast<float *>(sm.red));
+                                     reinterpret_cast<float *>(sm.red), p.st32 != 0);
             else
                 qk_tile<D, false>(st, p.Nq, t.tile, nullptr, sm.lut,
                                   p.q_fp4 + static_cast<size_t>(t.bh) * p.Npq * (D / 2),
-                                  p.q_sf + static_cast<size_t>(t.bh) * p.Npq * (D / 16));
+                                  p.q_sf + static_cast<size_t>(t.bh) * p.Npq * (D / 16), p.st32 != 0);
         } else if (t.kind == 1) {
             if constexpr (kI8)
-                v_tile_f16<D>(st, p.Np, t.tile, p.vt_fp4 + static_cast<size_t>(t.bh) * D * p.Np * 2);
+                v_tile_f16<D>(st, p.Np, t.tile, p.vt_fp4 + static_cast<size_t>(t.bh) * D * p.Np * 2, p.st32 != 0);
             else
                 v_tile<D>(st, p.Np, t.tile, sm.lut, p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
                           p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
@@ -617,11 +637,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if constexpr (kI8)
             qk_tile_i8<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean,
                                 reinterpret_cast<int8_t *>(p.k_fp4) + static_cast<size_t>(bh) * p.Np * D,
-                                p.k_scale + static_cast<size_t>(bh) * (p.Np / kTile), reinterpret_cast<float *>(sm.red));
+                                p.k_scale + static_cast<size_t>(bh) * (p.Np / kTile), reinterpret_cast<float *>(sm.red),
+                                p.st32 != 0);
         else
             qk_tile<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean, sm.lut,
                              p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
-                             p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16));
+                             p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16), p.st32 != 0);
         __syncthreads();  // stage s and neg_mean have been read by every thread
         if (threadIdx.x == 0 && i0 + n + kStages < i1) {
             fence_proxy_async_smem();

@@ -70,6 +70,7 @@ bool make_qkv_map(CUtensorMap *m, const void *base, int d, int N, int BH) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 int check_shape(int B, int H, int N, int d) {
     if (B < 1 || H < 1 || N < 1) return SA3_ERR_INVALID_ARG;
@@ -141,7 +142,7 @@ int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, in
     if ((rc = check_qkv(out)) != SA3_OK) return rc;
     const int64_t need = sa3_quant_workspace_bytes(B, H, Nkv, d);
     if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
-    sa3::QuantParams p;
+    sa3::QuantParams p = {};
     p.q_fp4 = static_cast<uint8_t *>(out->q_fp4);
     p.q_sf = static_cast<uint8_t *>(out->q_sf);
     p.k_fp4 = static_cast<uint8_t *>(out->k_fp4);
@@ -157,6 +158,7 @@ int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, in
     p.Npq = static_cast<int>(sa3_padded_len(Nq));
     p.chunk = static_cast<int>(sa3_kmean_chunk(Nkv));
     p.nchunk = static_cast<int>(sa3_kmean_nchunk(Nkv));
+    p.st32 = aligned32(p.q_fp4) && aligned32(p.k_fp4);
     CUtensorMap tq, tk, tv;
     if (!make_qkv_map(&tq, q, d, Nq, p.BH) || !make_qkv_map(&tk, k, d, Nkv, p.BH) ||
         !make_qkv_map(&tv, v, d, Nkv, p.BH))
@@ -192,6 +194,7 @@ int sa3_quantize_qkv_i8(const void *q, const void *k, const void *v, int B, int 
     p.Npq = static_cast<int>(sa3_padded_len(Nq));
     p.chunk = static_cast<int>(sa3_kmean_chunk(Nkv));
     p.nchunk = static_cast<int>(sa3_kmean_nchunk(Nkv));
+    p.st32 = aligned32(p.q_fp4) && aligned32(p.k_fp4) && aligned32(p.vt_fp4);
     CUtensorMap tq, tk, tv;
     if (!make_qkv_map(&tq, q, d, Nq, p.BH) || !make_qkv_map(&tk, k, d, Nkv, p.BH) ||
         !make_qkv_map(&tv, v, d, Nkv, p.BH))

@@ -28,6 +28,7 @@ struct QuantParams {
     int Npq;     // Nq rounded up to 128
     int nchunk;  // fp64 partial sums of K per (b, h)
     int chunk;   // tokens per partial sum
+    int st32;    // 1: the code outputs are 32-byte aligned, so tiles store 32-byte pieces in one instruction
 };
 
 struct AttnParams {

@@ -304,6 +304,13 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     return d;
 }
 
+// One 32-byte global store from eight words (address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 // ------------------------------------------------------------ conversions
 // E2M1 codes of 8 floats, packed: element 0 in bits [0,4), element 7 in
 // bits [28,32).  Round to nearest even, saturate at +-6.

@@ -101,3 +101,46 @@ def test_quantize_rejects_bad_arguments():
     with pytest.raises(sa3.Sa3Error) as e:
         sa3.quantize_qkv(q96, q96, q96)
     assert e.value.code == sa3.SA3_ERR_UNSUPPORTED
+
+
+def _offset16(t):
+    """A copy of t's shape and dtype whose storage starts 16 bytes past a
+    256-byte boundary: 16-byte aligned (the ABI's requirement), not 32."""
+    n = t.numel() * t.element_size()
+    buf = torch.empty(n + 256, dtype=torch.uint8, device=t.device)
+    base = (-buf.data_ptr()) % 256 + 16
+    out = buf[base:base + n].view(t.dtype).view(t.shape)
+    assert out.data_ptr() % 32 == 16
+    return out
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantize_outputs_only_16_byte_aligned(d):
+    """The tiles store 32-byte pieces in one instruction when every code
+    output is 32-byte aligned, else in 16-byte pieces: same bytes."""
+    import dataclasses
+    q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 300, "d": d})]
+    a = sa3.quantize_qkv(q, k, v)
+    b = sa3.empty_quantized(1, 2, 300, d)
+    b = dataclasses.replace(b, **{f: _offset16(getattr(b, f)) for f in ("q_fp4", "k_fp4", "vt_fp4")})
+    sa3.quantize_qkv(q, k, v, out=b)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    for f in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantize_i8_outputs_only_16_byte_aligned(d):
+    import dataclasses
+    q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 300, "d": d})]
+    a = sa3.quantize_qkv_i8(q, k, v)
+    b = sa3.empty_quantized_i8(1, 2, 300, d)
+    b = dataclasses.replace(b, **{f: _offset16(getattr(b, f)) for f in ("q_i8", "k_i8", "vt_f16")})
+    sa3.quantize_qkv_i8(q, k, v, out=b)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    for f in ("q_i8", "q_scale", "k_i8", "k_scale", "vt_f16", "k_mean"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
