@@ -367,6 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ff = pack2(f, f);
             const uint64_t nn = pack2(nm, nm);
             uint64_t acc = pack2(0.0f, 0.0f);
+            if (j > 0) {
+                if (!warp_wait(bars + kBarPvDone + i, (j - 1) & 1, abort_flag)) ok = false;
+                tc_fence_after();
+            }
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t ph[16];
@@ -377,10 +381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float p0 = ex2(lo2(t2)), p1 = ex2(hi2(t2));
                     acc = add2(acc, pack2(p0, p1));
                     ph[e] = f16x2(p0, p1);
-                }
-                if (half == 0 && j > 0) {
-                    if (!warp_wait(bars + kBarPvDone + i, (j - 1) & 1, abort_flag)) ok = false;
-                    tc_fence_after();
                 }
                 if (ok) {
 #pragma unroll
@@ -394,21 +394,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             l = alpha * l + (lo2(acc) + hi2(acc));
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-                uint32_t o[D / 64][32];
-#pragma unroll
-                for (int q = 0; q < D / 64; ++q) tmem_ld32(trow + tO + 32 * q, o[q]);
-                tmem_ld_wait();
                 const uint64_t aa = pack2(alpha, alpha);
 #pragma unroll
                 for (int q = 0; q < D / 64; ++q) {
-                    reg_fence32(o[q]);
+                    uint32_t o[32];
+                    tmem_ld32(trow + tO + 32 * q, o);
+                    tmem_ld_wait();
+                    reg_fence32(o);
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const uint64_t v = mul2(pack2(__uint_as_float(o[q][e]), __uint_as_float(o[q][e + 1])), aa);
-                        o[q][e] = __float_as_uint(lo2(v));
-                        o[q][e + 1] = __float_as_uint(hi2(v));
+                        const uint64_t v = mul2(pack2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa);
+                        o[e] = __float_as_uint(lo2(v));
+                        o[e + 1] = __float_as_uint(hi2(v));
                     }
-                    tmem_st32(trow + tO + 32 * q, o[q]);
+                    tmem_st32(trow + tO + 32 * q, o);
                 }
                 tmem_st_wait();
             }
