@@ -233,3 +233,30 @@ def test_max_in_first_block_matches_untiled_formula():
     assert rel_l2(out[rows], ref[rows]) <= 2e-3
     # rows whose maximum comes later see a different running max in block 0
     assert rel_l2(out[~rows], ref[~rows]) > 1e-3
+
+
+def _constant_v(q, seed=5):
+    """V constant over tokens, v_c = +-6 * 2^k_c per (b, h, channel): every
+    16-token block of V^T quantizes exactly (scale 2^k_c, code 6)."""
+    B, H, N, d = q.shape
+    g = np.random.default_rng(seed)
+    vc = g.choice([-1.0, 1.0], (B, H, 1, d)) * 6.0 * 2.0 ** g.integers(-3, 3, (B, H, 1, d))
+    return torch.from_numpy(np.broadcast_to(vc, (B, H, N, d)).copy()).to(torch.bfloat16), vc
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v_rows_are_v_times_one_factor(causal):
+    """With V^ = V constant over tokens, O_c = v_c * sum(P^) / sum(P): one
+    factor per row, and since the channels differ only by a sign and a power
+    of two, every rounding scales with them, so out / v is bit-identical
+    across channels.  Causal row 0 sees one key: P = 1, P^ = 6 * E4M3(1/6) =
+    1.03125.  The factor stays near 1 (P's FP4 rounding, averaged over the
+    row: between 0.92 and 1.09 on these inputs; bound 0.75 .. 1.25)."""
+    q, k, _ = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 300})
+    v, vc = _constant_v(q)
+    out = oracle.bf16_bits_to_f32(oracle.attn_fwd(oracle.quantize_qkv(q, k, v), 300, causal)).astype(np.float64)
+    ratio = out / vc
+    assert np.array_equal(ratio, np.broadcast_to(ratio[..., :1], ratio.shape))
+    assert (ratio > 0.75).all() and (ratio < 1.25).all()
+    if causal:
+        assert (ratio[:, :, 0] == 1.03125).all()

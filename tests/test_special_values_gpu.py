@@ -153,3 +153,30 @@ def test_quantize_i8_special_values_bit_exact(case):
         assert np.array_equal(g[f].view(np.uint32), r[f].view(np.uint32)), f
     if name.startswith("zeros"):
         assert not g["q_scale"].any() and not g["q_i8"].any() and not g["k_i8"].any()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["noncausal", "causal"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_attn_constant_v_rows_are_v_times_one_factor(d, causal):
+    """V constant over tokens with v_c = +-6 * 2^k_c (exact in FP4): each
+    output row is v times one factor, bit-identical across channels (the
+    tensor core sums every channel in the same order, and the channels
+    differ by a sign and a power of two), and equal to the oracle's."""
+    g = torch.Generator().manual_seed(d)
+    B, H, N = 1, 2, 300
+    q = torch.randn((B, H, N, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, H, N, d), generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(d)
+    vc = rng.choice([-1.0, 1.0], (B, H, 1, d)) * 6.0 * 2.0 ** rng.integers(-3, 3, (B, H, 1, d))
+    v = torch.from_numpy(np.broadcast_to(vc, (B, H, N, d)).copy()).to(torch.bfloat16)
+    qz, gq = _quantized(q, k, v)
+    out = sa3.attn_fwd(qz, causal=causal)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    ratio = out.double().cpu().numpy() / vc
+    assert np.array_equal(ratio, np.broadcast_to(ratio[..., :1], ratio.shape))
+    if causal:
+        assert (ratio[:, :, 0] == 1.03125).all()
+    ref = bits_to_f32(oracle.attn_fwd(gq, N, causal))
+    assert rel_l2(out.float().cpu().numpy(), ref) <= 2e-3
