@@ -23,6 +23,11 @@
  *     where N_p = N rounded up to a multiple of 128;
  *   - Q, K, V and the output are bf16, contiguous [B][H][N][d], 16-byte
  *     aligned;
+ *   - quantizer outputs need 16-byte alignment.  When all the code outputs
+ *     (q/k codes, V^T codes or FP16 V^T) are 32-byte aligned, as any
+ *     cudaMalloc or torch allocation is, the quantizer writes 32-byte pieces
+ *     in one store each, which is faster for the 8-bit variant.  The bytes
+ *     written are the same either way;
  *   - the library is thread-safe for concurrent calls on different streams
  *     as long as their workspaces differ.
  *
