@@ -362,8 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = ex2(__fsub_rn(m, m_new));
             // P = 2^(t - m'), fp32 row sum, fp16 P for P V; written to shared
             // memory in two halves of 32 keys (16-byte chunk c of this half,
-            // keys 8c .. 8c+7, at chunk c ^ (r % 8)), the first one once the
-            // previous P V has released the buffer
+            // keys 8c .. 8c+7, at chunk c ^ (r % 8)).  The previous P V must
+            // have released the buffer first; waiting for it before any P is
+            // computed keeps no half in registers across the wait
             const uint64_t ff = pack2(f, f);
             const uint64_t nn = pack2(nm, nm);
             uint64_t acc = pack2(0.0f, 0.0f);
