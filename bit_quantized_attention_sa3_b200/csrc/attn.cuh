@@ -618,7 +618,10 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     const bool two = p.p_pre_log2 != 0.0f;
     auto kernel = cross ? (two ? attn_fwd_kernel<D, true, true> : attn_fwd_kernel<D, true, false>)
                         : (two ? attn_fwd_kernel<D, false, true> : attn_fwd_kernel<D, false, false>);
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e = cross ? (two ? smem_attr_once<attn_fwd_kernel<D, true, true>>(C::kSmemBytes)
+                                 : smem_attr_once<attn_fwd_kernel<D, true, false>>(C::kSmemBytes))
+                          : (two ? smem_attr_once<attn_fwd_kernel<D, false, true>>(C::kSmemBytes)
+                                 : smem_attr_once<attn_fwd_kernel<D, false, false>>(C::kSmemBytes));
     if (e != cudaSuccess) return e;
     // Split the pairs of a last wave that would fill at most half of the SMs
     // into single-tile units (one CTA per SM).
@@ -626,8 +629,7 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     const int nqt = p.Npq / kBlk;
     q.npairs = (nqt + 1) / 2;
     const int total = q.npairs * p.BH;
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = sm_count();
     const int rem = total % nsm;
     const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;

@@ -473,14 +473,14 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
                      cudaStream_t stream) {
     using C = Cfg<D>;
     auto kernel = p.Nq != p.N ? attn8_fwd_kernel<D, true> : attn8_fwd_kernel<D, false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e = p.Nq != p.N ? smem_attr_once<attn8_fwd_kernel<D, true>>(C::kSmemBytes)
+                                : smem_attr_once<attn8_fwd_kernel<D, false>>(C::kSmemBytes);
     if (e != cudaSuccess) return e;
     AttnParams q = p;
     const int nqt = p.Npq / kBlk;
     q.npairs = (nqt + 1) / 2;
     const int total = q.npairs * p.BH;
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = sm_count();
     const int rem = total % nsm;
     const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;

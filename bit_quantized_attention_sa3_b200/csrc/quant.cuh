@@ -659,13 +659,11 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
                      cudaStream_t stream) {
     using C = QCfg<D>;
     if (p.nchunk > kMaxChunks || p.chunk % kTile != 0) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(quant_qvk_kernel<D, kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+    cudaError_t e = smem_attr_once<quant_qvk_kernel<D, kI8>>(C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(quant_k_kernel<D, kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = smem_attr_once<quant_k_kernel<D, kI8>>(C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = sm_count();
     const long long ntile = p.Np / kTile;
     const long long work_a = static_cast<long long>(p.BH) * (p.Npq / kTile + ntile) +
                              static_cast<long long>(p.BH) * p.nchunk;

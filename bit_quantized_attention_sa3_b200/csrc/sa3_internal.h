@@ -1,6 +1,7 @@
 // sa3_internal.h -- launch parameters shared by the host API and kernels.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -51,5 +52,38 @@ struct AttnParams {
     int npairs;        // Q-tile pairs per head (set by the launcher)
     int pair_units;    // work units that are pairs; the rest are single tiles
 };
+
+// Host: raise Kernel's dynamic shared memory limit once per device (the
+// attribute persists in the device's module), so that later calls -- those
+// recorded into a CUDA graph included -- make no attribute call.  Devices
+// 64 and up are set on every call.
+template <auto Kernel>
+inline cudaError_t smem_attr_once(int bytes) {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t{1} << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
+// Host: SM count of the current device (queried once per device; 148 if the
+// query fails).
+inline int sm_count() {
+    static std::atomic<int> cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 }  // namespace sa3
