@@ -58,6 +58,8 @@ _lib = None
 def lib() -> ctypes.CDLL:
     """Load libsa3.so (raises if it has not been built)."""
     global _lib
+    if _lib is not None:  # loaded: no lock on the per-call path
+        return _lib
     with _lock:
         if _lib is None:
             if not os.path.exists(LIB_PATH):

@@ -69,3 +69,17 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 8, 8, 96, None, None, 0, None) == 2
     assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 0, 64, 0, 0.0, 0, None, None) == 1
     assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 8, 64, 0, 0.0, 0, None, None) == 1
+
+
+def test_binding_loads_the_library_and_reports_its_version():
+    """The Python binding's own loader (no GPU needed to load or to ask the
+    version) sets every declared signature."""
+    import bit_quantized_attention_sa3_b200 as sa3
+    from bit_quantized_attention_sa3_b200 import build
+    build.build()
+    assert sa3.version().startswith("libsa3")
+    L = sa3.lib()
+    assert sa3.lib() is L
+    for name in _declared():
+        if name not in ("sa3_selftest_wait_timeout", "sa3_quantize_qkv_noalloc", "sa3_version"):
+            assert getattr(L, name).argtypes, name  # ctypes leaves argtypes None unless set
