@@ -54,3 +54,24 @@ def test_bench_cli_rejects_world_mismatch(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "1")
     with pytest.raises(SystemExit):
         bench.dist_init(2)
+
+
+def test_bench_reference_arm_under_torchrun_two_ranks():
+    """bench.py itself, launched as the multi-GPU runs are (torchrun, one
+    process per rank), on the reference arm (CPU oracle; gloo on a host
+    without CUDA): rank 0 prints the one JSON line for the whole job, the
+    other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.join(root, "bench.py"),
+           "--gpus", "2", "--impl", "reference", "--workload", "tiny_b1h2n256d64", "--steps", "2", "--warmup", "1"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
