@@ -69,6 +69,13 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.sa3_quantize_qkv_lens(16, 16, 16, 1, 1, 8, 8, 96, None, None, 0, None) == 2
     assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 0, 64, 0, 0.0, 0, None, None) == 1
     assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, 8, 64, 0, 0.0, 0, None, None) == 1
+    # size limit B*H*N_p*d/2 < 2^31: exactly at it -> unsupported; one tile
+    # below passes the shape check and fails on the null pointers instead
+    at = 1 << 25  # N_p * 128 / 2 = 2^31 with B = H = 1, d = 128
+    assert lib.sa3_quantize_qkv(16, 16, 16, 1, 1, at, 128, None, None, 0, None) == 2
+    assert lib.sa3_attn_fwd(None, 1, 1, at, 128, 0, 0.0, None, None) == 2
+    assert lib.sa3_attn_fwd(None, 1, 1, at - 128, 128, 0, 0.0, None, None) == 1
+    assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, at, 128, 0, 0.0, 0, None, None) == 2
 
 
 def test_binding_loads_the_library_and_reports_its_version():

@@ -165,3 +165,33 @@ def test_causal_row0_matches_oracle_exactly():
     got = out[:, :, 0].float().cpu().numpy()
     want = bits_to_f32(ref[:, :, 0])
     assert np.all(np.abs(got - want) <= 2.0 ** -7 * np.abs(want))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["noncausal", "causal"])
+def test_long_sequence_131072_tokens(causal):
+    """Four times the longest workload: B=1, H=2, N=131072, d=128 (its
+    distribution).  Quantization bit-exact on the whole tensors; attention
+    against the oracle on the first, the last and one seeded block of each
+    head (the last block's causal rows see all 131072 keys)."""
+    name, over = "longctx_b1h32n32768d128_causal", {"H": 2, "N": 131072}
+    q, k, v = sa3_inputs.make_qkv(name, shape_override=over)
+    B, H, N, d = q.shape
+    qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
+    out = sa3.attn_fwd(qz, causal=causal)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    canon = _canonical(qz, B, H, N, d)
+    if not causal:  # the quantized operands do not depend on the mask: compare once
+        r = oracle.quantize_qkv(q, k, v)
+        for f in ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf"):
+            assert np.array_equal(canon[f], r[f]), f
+        assert np.array_equal(qz.k_mean.cpu().numpy().view(np.uint32), r["k_mean"].view(np.uint32))
+    nqb = N // 128
+    units = [(bh, qb) for bh in range(B * H) for qb in (0, nqb - 1, 517)]
+    ref = bits_to_f32(oracle.attn_fwd(canon, N, causal, units=units)).reshape(B * H, N, d)
+    got = out.float().cpu().numpy().reshape(B * H, N, d)
+    assert np.isfinite(got).all()
+    for bh, qb in units:
+        rows = slice(qb * 128, qb * 128 + 128)
+        assert rel_l2(got[bh, rows], ref[bh, rows]) <= TOL, (bh, qb)
