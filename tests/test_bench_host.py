@@ -47,3 +47,55 @@ def test_make_inputs_shapes_and_prefix(bench, Nq):
     if Nq <= w.N:
         q0, k0, v0 = sa3_inputs.make_qkv(w, seed=0)
         assert (q == q0[:, :, :Nq]).all() and (k == k0).all() and (v == v0).all()
+
+
+REQUIRED = {"metric": str, "value": (int, float), "unit": str, "n_gpus": int, "steps": int, "warmup": int,
+            "ms_per_step": (int, float), "higher_is_better": bool, "scaling": str, "dtype": str, "data": str,
+            "config": dict, "e2e": dict}
+
+
+def _check_line(line):
+    for k, t in REQUIRED.items():
+        assert k in line and isinstance(line[k], t), k
+    assert "vs_baseline" in line and line["vs_baseline"] is None
+    assert line["config"]["workload"] and line["value"] > 0
+    for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert k in line["e2e"], k
+
+
+def test_reference_arm_prints_the_contract_line():
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "tiny_b1h2n256d64", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    _check_line(line)
+    assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+
+
+@pytest.mark.gpu
+def test_gpu_arm_prints_the_contract_line():
+    """The benchmark's own arm on the headline workload, briefly: every key of
+    the line, the roofline object, clocks and the launch count."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "3", "--warmup", "3",
+                        "--skip-cpu-baseline"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    _check_line(line)
+    roof = line["roofline"]
+    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s" and 0 < roof["frac"] < 1.5
+    assert abs(roof["achieved"] / roof["peak"] - roof["frac"]) < 1e-3
+    assert line["gpu_launches"] == 3 * line["steps"]
+    assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(line["clocks"])
+    assert line["e2e"]["h2d_bytes_per_step"] == 3 * 2 * 16 * 4096 * 128 * 2
