@@ -7,6 +7,16 @@ library is missing or a call fails, an exception is raised.
 
     qz = quantize_qkv(q, k, v)          # K smoothing + FP4 microscaling
     out = attn_fwd(qz, causal=False)    # FP4 attention, bf16 out
+    out = sa3_attention(q, k, v)        # both in one call
+
+    q8 = quantize_qkv_i8(q, k, v)       # 8-bit variant: INT8 Q, K; FP16 V^T
+    out, lse = attn_fwd_i8(q8, causal=True, lse=True)   # training forward
+
+q may be shorter or longer than k and v (the *_lens calls).  Every call is
+asynchronous on the current torch stream (or ``stream=``); buffers can be
+passed in (``out=``, ``workspace=``) so that a step allocates nothing and can
+be recorded into a CUDA graph.  ``device_status()`` synchronizes and reports
+whether a bounded device wait gave up.
 """
 from __future__ import annotations
 
