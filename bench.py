@@ -15,6 +15,12 @@ synchronize around the K timed steps; multi-GPU runs take the maximum
 over ranks and report the whole-job rate (every rank runs its own batch:
 weak scaling, no data-path collective).
 
+Options: --variant i8 times the 8-bit variant (INT8 QK^T, FP16 P V) and
+i8_train its training forward (also writes the per-row log-sum-exp);
+--workload picks another seeded workload; --nq gives Q fewer or more tokens
+than K and V (ops then count the (query, key) pairs the mask leaves);
+--p-two-level times the two-level P recipe.
+
 --impl reference runs the CPU oracle (oracle/) as it stands on the host
 cores, on a bounded sample of the same workload, and prints the same line
 with "impl": "reference".
