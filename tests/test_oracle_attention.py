@@ -260,3 +260,25 @@ def test_constant_v_rows_are_v_times_one_factor(causal):
     assert (ratio > 0.75).all() and (ratio < 1.25).all()
     if causal:
         assert (ratio[:, :, 0] == 1.03125).all()
+
+
+@pytest.mark.parametrize("Nq,Nkv,causal,sm", [(300, 300, False, None), (300, 300, True, None), (77, 300, True, 0.3),
+                                              (300, 77, False, None), (129, 1, True, None)])
+def test_exact_attention_matches_torch_sdpa(Nq, Nkv, causal, sm):
+    """The fp64 reference against PyTorch's scaled_dot_product_attention in
+    float64 on the same bf16 inputs.  The causal mask is passed explicitly,
+    bottom-right aligned (query r sees keys 0 .. r + Nkv - Nq); rows that see
+    no key are left out (the oracle gives them 0, the library routine NaN)."""
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": max(Nq, Nkv)})
+    q, k, v = q[:, :, :Nq].contiguous(), k[:, :, :Nkv].contiguous(), v[:, :, :Nkv].contiguous()
+    d = q.shape[-1]
+    got = oracle.attn_exact(q, k, v, causal, sm_scale=sm)
+    vis = torch.ones((Nq, Nkv), dtype=torch.bool)
+    if causal:
+        vis = torch.arange(Nkv)[None, :] <= torch.arange(Nq)[:, None] + (Nkv - Nq)
+    scale = float(np.float32((1.0 / np.sqrt(d)) if sm is None else sm))  # the oracle takes sm_scale as fp32
+    want = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double(), v.double(), attn_mask=vis, scale=scale).numpy()
+    live = vis.any(dim=1).numpy()
+    np.testing.assert_allclose(got[:, :, live], want[:, :, live], rtol=1e-12, atol=1e-12)
+    assert not got[:, :, ~live].any()
