@@ -282,3 +282,31 @@ def test_exact_attention_matches_torch_sdpa(Nq, Nkv, causal, sm):
     live = vis.any(dim=1).numpy()
     np.testing.assert_allclose(got[:, :, live], want[:, :, live], rtol=1e-12, atol=1e-12)
     assert not got[:, :, ~live].any()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_units_equal_the_full_computation(causal):
+    """The full-size GPU tests compare only sampled (head, Q block) units
+    against the oracle, so the unit path must give exactly the rows of the
+    full computation and leave every other row untouched: FP4, 8-bit (with
+    the log-sum-exp) and exact attention."""
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 300, "H": 3})
+    B, H, N, d = q.shape
+    units = [(0, 2), (2, 0), (1, 1)]
+    rows = np.zeros((B * H, N), bool)
+    for bh, qb in units:
+        rows[bh, qb * 128: min(N, qb * 128 + 128)] = True
+    rows = rows.reshape(B, H, N)
+
+    qz = oracle.quantize_qkv(q, k, v)
+    full, part = oracle.attn_fwd(qz, N, causal), oracle.attn_fwd(qz, N, causal, units=units)
+    assert np.array_equal(part[rows], full[rows]) and not part[~rows].any()
+
+    q8 = oracle.quantize_qkv_i8(q, k, v)
+    f8, fl = oracle.attn_fwd_i8(q8, N, causal, return_lse=True)
+    p8, pl = oracle.attn_fwd_i8(q8, N, causal, units=units, return_lse=True)
+    assert np.array_equal(p8[rows], f8[rows]) and not p8[~rows].any()
+    assert np.array_equal(pl[rows], fl[rows]) and np.isnan(pl[~rows]).all()
+
+    ex, pe = oracle.attn_exact(q, k, v, causal), oracle.attn_exact(q, k, v, causal, units=units)
+    assert np.array_equal(pe[rows], ex[rows]) and not pe[~rows].any()
