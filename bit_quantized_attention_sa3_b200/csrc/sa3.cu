@@ -77,7 +77,6 @@ int check_shape(int B, int H, int N, int d) {
     if (d != 64 && d != 128) return SA3_ERR_UNSUPPORTED;
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int64_t Np = sa3_padded_len(N);
-    if (BH > 65535) return SA3_ERR_UNSUPPORTED;  // grid y
     if (BH * Np * d / 2 >= (int64_t(1) << 31) || BH * Np >= (int64_t(1) << 31)) return SA3_ERR_UNSUPPORTED;
     return SA3_OK;
 }

@@ -195,3 +195,27 @@ def test_long_sequence_131072_tokens(causal):
     for bh, qb in units:
         rows = slice(qb * 128, qb * 128 + 128)
         assert rel_l2(got[bh, rows], ref[bh, rows]) <= TOL, (bh, qb)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["noncausal", "causal"])
+def test_many_heads_beyond_65535(causal):
+    """B*H = 66000 short heads (N = 40, d = 64): grids are one-dimensional,
+    so B*H is bounded only by the size limit.  Heads on both sides of
+    65536 and the last one are compared with the oracle run on their slice
+    (quantization and attention of one head do not depend on the others)."""
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"B": 2, "H": 33000, "N": 40})
+    B, H, N, d = q.shape
+    qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
+    out = sa3.attn_fwd(qz, causal=causal)
+    torch.cuda.synchronize()
+    assert sa3.device_status() == sa3.SA3_OK
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    codes = qz.k_fp4.cpu().numpy()
+    for bh in (0, 65535, 65536, B * H - 1):
+        b, h = divmod(bh, H)
+        sl = slice(b, b + 1), slice(h, h + 1)
+        r = oracle.quantize_qkv(q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous())
+        assert np.array_equal(codes[b, h], r["k_codes"][0, 0]), bh
+        ref = bits_to_f32(oracle.attn_fwd(r, N, causal))[0, 0]
+        assert rel_l2(bits_to_f32(got[b, h]), ref) <= TOL, bh
