@@ -29,7 +29,12 @@
  *     in one store each, which is faster for the 8-bit variant.  The bytes
  *     written are the same either way;
  *   - the library is thread-safe for concurrent calls on different streams
- *     as long as their workspaces differ.
+ *     as long as their workspaces differ;
+ *   - the first call of each kernel on a device sets that kernel's
+ *     attributes, once.  Make it outside stream capture.  After it, the
+ *     calls only enqueue kernels, with no allocation, synchronization or
+ *     attribute call, so they can be recorded into a CUDA graph (stream
+ *     capture) and replayed with new inputs in the same buffers.
  *
  * Error behaviour: arguments are checked before any launch; a bad argument
  * returns SA3_ERR_INVALID_ARG (null pointer, misalignment, non-positive
