@@ -154,6 +154,13 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v,
  * out = bf16_RN(O / l).  ("Online normalizer calculation for softmax" and
  * the FlashAttention papers, in the SageAttention3 reference list.)
  *
+ * Accuracy: the recipe above is followed step by step, but not to the bit.
+ * The exponentials use the hardware's approximate exp2.  1/s is folded into
+ * the exponent: y = 2^(t - m' + log2(1/s)), rounded at the size of m'.
+ * Tensor-core sums run in their own order.  So a P code may differ from
+ * the recipe's where the value sits at a rounding boundary.  Outputs stay
+ * within relative L2 2e-3 of the step-by-step recipe.
+ *
  * in       : quantized operands from sa3_quantize_qkv for the same shape.
  * causal   : 0 or 1 (mask col > row, rows and columns both from 0).
  * sm_scale : softmax scale; <= 0 selects 1/sqrt(d).
