@@ -1,0 +1,78 @@
+// Host-side check of the quantizer's static schedule (SchedA in quant.cuh),
+// run by tests/test_quant_schedule.py: for every listed shape and grid size,
+// each Q tile, V tile and K tile is handed out exactly once, every K tile
+// belongs to the chunk it is reported in, every chunk is flushed exactly
+// once (its last tile), no job is out of range, and no CTA receives more
+// than the average plus one chunk of tiles.  Only host code runs.
+#include "quant.cuh"
+
+#include <cstdio>
+#include <vector>
+
+int main() {
+    long long checked = 0;
+    for (int BH : {1, 2, 3, 7, 30, 32, 128, 151})
+        for (int N : {1, 100, 128, 129, 300, 1000, 4096, 8192, 17776, 32768})
+            for (int Nq : {N, 1, 77, 2000}) {
+                const int ntile = (N + 127) / 128;
+                const int ntq = (Nq + 127) / 128;
+                const int chunk = 512 * (((N + 511) / 512 + 15) / 16);  // sa3_kmean_chunk
+                const int nchunk = (N + chunk - 1) / chunk;
+                const int tpc = chunk / 128;
+                for (int G : {1, 2, 5, 37, 148, 296}) {
+                    const long long work = (long long)BH * (ntile + ntq) + (long long)BH * nchunk;
+                    const int Gx = work < G ? (int)work : G;
+                    std::vector<int> q(BH * ntq, 0), v(BH * ntile, 0), k(BH * ntile, 0), last(BH * nchunk, 0);
+                    int maxload = 0;
+                    for (int g = 0; g < Gx; ++g) {
+                        sa3::quant::SchedA s;
+                        s.init(BH, ntq, ntile, nchunk, tpc, g, Gx);
+                        sa3::quant::TileJob t;
+                        int load = 0;
+                        while (s.next(t)) {
+                            ++load;
+                            if (t.bh < 0 || t.bh >= BH || t.tile < 0 || t.tile >= (t.kind == 0 ? ntq : ntile)) {
+                                printf("job out of range: BH=%d N=%d Nq=%d G=%d\n", BH, N, Nq, Gx);
+                                return 1;
+                            }
+                            if (t.kind == 0) {
+                                q[t.bh * ntq + t.tile]++;
+                            } else if (t.kind == 1) {
+                                v[t.bh * ntile + t.tile]++;
+                            } else {
+                                k[t.bh * ntile + t.tile]++;
+                                if (t.tile / tpc != t.chunk) {
+                                    printf("K tile outside its chunk: BH=%d N=%d G=%d\n", BH, N, Gx);
+                                    return 1;
+                                }
+                                if (t.last) last[t.bh * nchunk + t.chunk]++;
+                            }
+                        }
+                        if (load > maxload) maxload = load;
+                    }
+                    for (int i = 0; i < BH * ntq; ++i)
+                        if (q[i] != 1) {
+                            printf("Q tile %d handed out %d times: BH=%d Nq=%d G=%d\n", i, q[i], BH, Nq, Gx);
+                            return 1;
+                        }
+                    for (int i = 0; i < BH * ntile; ++i)
+                        if (v[i] != 1 || k[i] != 1) {
+                            printf("V/K tile %d: %d / %d times: BH=%d N=%d G=%d\n", i, v[i], k[i], BH, N, Gx);
+                            return 1;
+                        }
+                    for (int i = 0; i < BH * nchunk; ++i)
+                        if (last[i] != 1) {
+                            printf("chunk %d flushed %d times: BH=%d N=%d G=%d\n", i, last[i], BH, N, Gx);
+                            return 1;
+                        }
+                    const double avg = (double)((long long)BH * (2LL * ntile + ntq)) / Gx;
+                    if (Gx > 2 && maxload > avg + tpc + 2) {
+                        printf("imbalance: BH=%d N=%d Nq=%d G=%d max %d avg %.1f\n", BH, N, Nq, Gx, maxload, avg);
+                        return 1;
+                    }
+                    ++checked;
+                }
+            }
+    printf("ok %lld cases\n", checked);
+    return 0;
+}
