@@ -186,6 +186,78 @@ def profiled_traffic(kernel_src: str, profile: str):
     return None
 
 
+def fp4_peak_probe(sa3, dev, iters=16384):
+    """Block-scaled FP4 tensor-core rate on this GPU (sa3_probe_fp4_mma: one
+    CTA per SM, M=128, K=64, N=128 and N=256), timed with CUDA events on the
+    launching stream; best of 3 per shape.  Every run's accumulators are
+    checked to hold 64*iters (the tensor core did every MMA)."""
+    ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    res = {}
+    for n in (128, 256):
+        sa3.probe_fp4_mma(n=n, iters=256, device=dev)  # warm-up
+        best = None
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            out = sa3.probe_fp4_mma(n=n, iters=iters, device=dev)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if not torch.all(out == 64.0 * iters):
+                raise RuntimeError(f"FP4 MMA probe (N={n}) accumulated the wrong values")
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        res[f"n{n}_tops"] = round(2.0 * 128 * n * 64 * iters * ctas / (best * 1e-3) / 1e12, 1)
+    res["tops"] = max(res["n128_tops"], res["n256_tops"])
+    res["how"] = (f"sa3_probe_fp4_mma: {ctas} CTAs x {iters} tcgen05.mma.kind::mxf4nvf4.block_scale "
+                  f"(M=128, K=64), best of 3 per N, CUDA events")
+    return res
+
+
+def accuracy_sample(w, q, k, v, out, causal, two=False, nunits=6):
+    """The output's accuracy on a seeded sample of (head, Q block) units: the
+    oracle quantizes those heads itself and attends on its own operands
+    (worst per-block rel-L2 of the GPU output against it), and the fp64
+    exact attention of the bf16 inputs gives the cosines of both."""
+    import numpy as np
+    import oracle
+    Nq, N = q.shape[2], k.shape[2]
+    nqb = (Nq + 127) // 128
+    rng = np.random.default_rng(1)
+    units = sorted({(0, 0), (w.B * w.H - 1, nqb - 1)} |
+                   {(int(rng.integers(w.B * w.H)), int(rng.integers(nqb))) for _ in range(nunits - 2)})
+    heads = sorted({bh for bh, _ in units})
+    pos = {bh: i for i, bh in enumerate(heads)}
+    sub = [(pos[bh], qb) for bh, qb in units]
+
+    def hd(t):
+        B, H, n, d = t.shape
+        return t.reshape(B * H, n, d)[heads].reshape(1, len(heads), n, d).contiguous()
+    qs, ks, vs = hd(q), hd(k), hd(v)
+    rq = oracle.quantize_qkv(qs, ks, vs)
+    ref = oracle.bf16_bits_to_f32(oracle.attn_fwd(rq, Nq, causal, units=sub, p_two_level=two))[0]
+    ex = oracle.attn_exact(qs, ks, vs, causal, units=sub)[0]
+    got = out.float().cpu().numpy().reshape(w.B * w.H, Nq, w.d)[heads]
+    live = (np.arange(Nq) + (N - Nq) >= 0) if causal else np.ones(Nq, bool)
+    worst, gs, rs, es = 0.0, [], [], []
+    for h, qb in sub:
+        rows = np.arange(qb * 128, min(Nq, qb * 128 + 128))
+        rows = rows[live[rows]]
+        if rows.size == 0:
+            continue
+        g, r, e = (a[h, rows].astype(np.float64) for a in (got, ref, ex))
+        worst = max(worst, float(np.linalg.norm(g - r) / np.linalg.norm(r)))
+        gs.append(g.ravel())
+        rs.append(r.ravel())
+        es.append(e.ravel())
+    g, r, e = np.concatenate(gs), np.concatenate(rs), np.concatenate(es)
+
+    def cos(a, b):
+        return float(a @ b / np.sqrt((a @ a) * (b @ b)))
+    return {"rel_l2_vs_oracle_worst_block": float(f"{worst:.3e}"), "cosine_vs_exact": round(cos(g, e), 5),
+            "oracle_cosine_vs_exact": round(cos(r, e), 5),
+            "sample": f"{len(units)} (head, 128-row Q block) units; the oracle quantizes those heads itself"}
+
+
 def attn_ops(w, Nq):
     """4*d per visible (query, key) pair: the workload's own count (4*B*H*N^2*d,
     halved for causal) when Nq == N, else the exact count of pairs that the
@@ -335,6 +407,7 @@ def run_sa3(args, rank, world, local):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
 
+    probe = None if i8 else fp4_peak_probe(sa3, dev)
     t_step = gmax(sum(step_ms) / len(step_ms))
     t_quant = gmax(sum(quant_ms) / len(quant_ms))
     t_attn = gmax(sum(attn_ms) / len(attn_ms))
@@ -354,8 +427,10 @@ def run_sa3(args, rank, world, local):
         dtype = "int8 QK^T (fp32 scale per 128-token tile), fp16 P V, fp32 accumulate"
         kernel, traffic = "attn8_fwd_kernel<%d>" % d, None
     else:
-        peak = pk["bf16_tflops"] * FP4_PER_BF16
-        peak_src = f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"
+        peak = probe["tops"]
+        peak_src = (f"measured in this run: {probe['how']} (N=128 {probe['n128_tops']}, "
+                    f"N=256 {probe['n256_tops']} TOPS)")
+        peak_rule = pk["bf16_tflops"] * FP4_PER_BF16
         qk_bytes = rd + B * H * d * (Npq + 2 * Np) // 2 + B * H * d * (Npq + 2 * Np) // 16
         dtype = "fp4-e2m1 (ue4m3 scales, fp32 accumulate)"
         kernel = "attn_fwd_kernel<%d>" % d
@@ -395,12 +470,18 @@ def run_sa3(args, rank, world, local):
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
+    if not i8:
+        line["roofline"]["peak_bf16x4"] = round(peak_rule, 1)
+        line["roofline"]["frac_of_bf16x4"] = round(achieved / peak_rule, 4)
+        line["roofline"]["peak_bf16x4_source"] = f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"
     if Nq != N:
         line["config"]["Nq"] = Nq
         line["config"]["ops"] = "4*d per (query, key) pair the mask leaves"
     if two:
         line["config"]["p_two_level"] = True
     if world == 1 and not args.skip_cpu_baseline:
+        if not i8:
+            line["accuracy"] = accuracy_sample(w, q_h, k_h, v_h, out, causal, two=two)
         line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8, train=train, two=two)
     print(json.dumps(line), flush=True)
 
@@ -458,19 +539,25 @@ def run_reference(args, rank, world):
     w = sa3_inputs.WORKLOADS[args.workload]
     Nq = args.nq or w.N
     q, k, v = make_inputs(w, Nq, seed=0)
-    per_step = []
+    per_step, wall = [], []
     budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
     i8, train = args.variant in ("i8", "i8_train"), args.variant == "i8_train"
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         cb = cpu_baseline(w, q, k, v, budget_s=budget, i8=i8, train=train, two=bool(args.p_two_level))
         if i >= args.warmup:
             per_step.append(cb)
+            wall.append(time.perf_counter() - t0)
     vals = [c["value"] for c in per_step]
     value = statistics.mean(vals)
     last = per_step[-1]
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(attn_ops(w, Nq) / (value * 1e12) * 1e3, 3),
+        "ms_per_step_kind": ("extrapolated: the time the oracle would take for one whole step, from full "
+                             "quantization plus a timed sample of Q blocks; each sampled step took "
+                             "sampled_ms_per_step of wall time"),
+        "sampled_ms_per_step": round(1e3 * statistics.mean(wall), 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)",
         "data": "synthetic (seeded, sa3_inputs.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,

@@ -164,15 +164,22 @@ __device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N
 
 // One staged 128-token tile of V, quantized transposed: blocks of 16 tokens
 // per channel.  Thread: channel pair (2cp, 2cp+1), 16-token blocks
-// g*D/64 .. g*D/64 + D/64 - 1.
-template <int D>
-__device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int Np, int tile,
-                                       const float *__restrict__ rcp_lut, uint8_t *__restrict__ vt,
-                                       uint8_t *__restrict__ vsf) {
+// g*D/64 .. g*D/64 + D/64 - 1.  kSmooth: -mean of V per channel is added to
+// tokens t < N (the fp32 subtraction V - mean, as for K); padding tokens
+// stay 0.
+template <int D, bool kSmooth>
+__device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int N, int Np, int tile,
+                                       const float *__restrict__ neg_mean, const float *__restrict__ rcp_lut,
+                                       uint8_t *__restrict__ vt, uint8_t *__restrict__ vsf) {
     constexpr int kPairs = D / 2;
     constexpr int kTbpt = D / 64;  // 16-token blocks per thread (2 or 1)
     const int cp = static_cast<int>(threadIdx.x) % kPairs;
     const int g = static_cast<int>(threadIdx.x) / kPairs;
+    float nm0 = 0.0f, nm1 = 0.0f;
+    if constexpr (kSmooth) {
+        nm0 = neg_mean[2 * cp];
+        nm1 = neg_mean[2 * cp + 1];
+    }
     uint32_t c0[2 * kTbpt], c1[2 * kTbpt];
     uint32_t s0 = 0, s1 = 0;
 #pragma unroll
@@ -186,6 +193,11 @@ __device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int Np
             const uint32_t w1 = *reinterpret_cast<const uint32_t *>(stage + tile_off(r + 1, 2 * cp));
             x0[k / 2] = pack2(bf16_lo(w0), bf16_lo(w1));
             x1[k / 2] = pack2(bf16_hi(w0), bf16_hi(w1));
+            if constexpr (kSmooth) {
+                const int t = tile * kTile + r;  // tokens t, t+1 (channel pairs 2cp, 2cp+1)
+                x0[k / 2] = add2(x0[k / 2], pack2(t < N ? nm0 : 0.0f, t + 1 < N ? nm0 : 0.0f));
+                x1[k / 2] = add2(x1[k / 2], pack2(t < N ? nm1 : 0.0f, t + 1 < N ? nm1 : 0.0f));
+            }
         }
         const uint32_t sc0 = scale_code(amax16(x0));
         const uint32_t sc1 = scale_code(amax16(x1));
@@ -381,35 +393,37 @@ __device__ __forceinline__ void ksum_flush(double (&acc)[8], double *red, double
 // ------------------------------------------------------------- schedule
 // Work of the first launch for CTA g of G: a contiguous range of the Q and
 // V tiles (Q tiles of every (b, h) first, then V; Q and V may have different
-// token counts), then the K chunks
-// g, g+G, g+2G, ... one tile at a time.  The Q/V ranges are sized so that
-// every CTA ends up with about the same number of tiles: CTAs holding one
-// K chunk more (the first nK % G) take tpc fewer Q/V tiles.
+// token counts), then the column-sum chunks g, g+G, g+2G, ... one tile at a
+// time: K's chunks, then (V smoothing) V's, whose tiles then go to the
+// second launch instead.  The Q/V ranges are sized so that every CTA ends
+// up with about the same number of tiles: CTAs holding one chunk more (the
+// first nK % G) take tpc fewer Q/V tiles.
 struct TileJob {
-    int kind;  // 0 = Q, 1 = V, 2 = K column sums
+    int kind;  // 0 = Q, 1 = V, 2 = K column sums, 3 = V column sums
     int bh;
     int tile;
-    int chunk;      // K: chunk of the tile
-    bool last;      // K: last tile of its chunk
+    int chunk;      // sums: chunk of the tile
+    bool last;      // sums: last tile of its chunk
 };
 
 struct SchedA {
-    int ntile_q, ntile, nchunk, tpc, nqk;  // nqk = BH * ntile_q (Q tiles; V tiles follow)
+    int ntile_q, ntile, nchunk, tpc, nqk, nsum;  // nqk = BH * ntile_q (Q tiles; V tiles follow)
     int j, je;                    // Q/V tiles [j, je)
-    int ki, nK, G;                // next K chunk item, items, stride
-    int kbh, kch, kt, kt_end;     // current K chunk and its tiles [kt, kt_end)
+    int ki, nK, G;                // next chunk item, items, stride
+    int kkind, kbh, kch, kt, kt_end;  // current chunk (2 = K, 3 = V) and its tiles [kt, kt_end)
 
-    __host__ __device__ void init(int BH, int ntile_q_, int ntile_, int nchunk_, int tpc_, int g, int G_) {
+    __host__ __device__ void init(int BH, int ntile_q_, int ntile_, int nchunk_, int tpc_, int g, int G_,
+                                  bool vsmooth = false) {
         ntile_q = ntile_q_;
         ntile = ntile_;
         nchunk = nchunk_;
         tpc = tpc_;
         nqk = BH * ntile_q;
         G = G_;
-        nK = BH * nchunk;
-        const int nqv = nqk + BH * ntile;
-        const int a = nK / G, r = nK % G;
-        (void)a;
+        nsum = BH * nchunk;
+        nK = nsum * (vsmooth ? 2 : 1);
+        const int nqv = nqk + (vsmooth ? 0 : BH * ntile);
+        const int r = nK % G;
         long long q_hi = (static_cast<long long>(nqv) + static_cast<long long>(r) * tpc + G - 1) / G;
         long long q_lo = q_hi - tpc;
         if (q_lo < 0) {
@@ -422,6 +436,7 @@ struct SchedA {
         je = static_cast<int>(pre + cnt < nqv ? pre + cnt : nqv);
         ki = g;
         kt = kt_end = 0;
+        kkind = 2;
         kbh = kch = 0;
     }
     __host__ __device__ bool next(TileJob &t) {
@@ -439,13 +454,15 @@ struct SchedA {
         }
         if (kt >= kt_end) {
             if (ki >= nK) return false;
-            kbh = ki / nchunk;
-            kch = ki % nchunk;
+            kkind = ki < nsum ? 2 : 3;
+            const int kk = ki < nsum ? ki : ki - nsum;
+            kbh = kk / nchunk;
+            kch = kk % nchunk;
             kt = kch * tpc;
             kt_end = kt + tpc < ntile ? kt + tpc : ntile;
             ki += G;
         }
-        t.kind = 2;
+        t.kind = kkind;
         t.bh = kbh;
         t.tile = kt;
         t.chunk = kch;
@@ -522,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const SmemPtrs sm = smem_setup<D>(smem_raw);
     SchedA prod, cons;
     prod.init(p.BH, p.Npq / kTile, p.Np / kTile, p.nchunk, p.chunk / kTile, static_cast<int>(blockIdx.x),
-              static_cast<int>(gridDim.x));
+              static_cast<int>(gridDim.x), p.vsmooth != 0);
     cons = prod;
     const uint64_t pol_once = l2_policy_evict_first();
     const uint64_t pol_k = l2_policy_evict_normal();
@@ -530,8 +547,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     auto issue_next = [&](int s) {
         TileJob t;
         if (!prod.next(t)) return;
-        const CUtensorMap *m = t.kind == 0 ? &tm_q : (t.kind == 1 ? &tm_v : &tm_k);
-        ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, m, t.bh, t.tile, t.kind == 2 ? pol_k : pol_once);
+        const CUtensorMap *m = t.kind == 0 ? &tm_q : (t.kind == 2 ? &tm_k : &tm_v);
+        // column-summed K (and V) tiles are read again by the second launch
+        ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, m, t.bh, t.tile, t.kind >= 2 ? pol_k : pol_once);
         ++issued;
     };
     if (threadIdx.x == 0) {
@@ -564,14 +582,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if constexpr (kI8)
                 v_tile_f16<D>(st, p.Np, t.tile, p.vt_fp4 + static_cast<size_t>(t.bh) * D * p.Np * 2, p.st32 != 0);
             else
-                v_tile<D>(st, p.Np, t.tile, sm.lut, p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
-                          p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
+                v_tile<D, false>(st, p.N, p.Np, t.tile, nullptr, sm.lut,
+                                 p.vt_fp4 + static_cast<size_t>(t.bh) * D * (p.Np / 2),
+                                 p.vt_sf + static_cast<size_t>(t.bh) * p.Np * 8);
         } else {
             ksum_tile<D>(st, acc);
         }
         __syncthreads();  // stage s has been read by every thread
-        if (t.kind == 2 && t.last)
-            ksum_flush<D>(acc, sm.red, p.part + (static_cast<size_t>(t.bh) * p.nchunk + t.chunk) * D);
+        if (t.kind >= 2 && t.last)
+            ksum_flush<D>(acc, sm.red,
+                          (t.kind == 2 ? p.part : p.vpart) + (static_cast<size_t>(t.bh) * p.nchunk + t.chunk) * D);
         if (threadIdx.x == 0) {
             fence_proxy_async_smem();
             issue_next(s);
@@ -580,53 +600,64 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (!ok && threadIdx.x == 0) ring_drain(sm.full, n, issued);
 }
 
-// Second launch: K tiles [g*T/G, (g+1)*T/G) of the T = BH * ntile tiles,
-// smoothed by the mean of their (b, h) and quantized.
+// Second launch: tiles [g*T/G, (g+1)*T/G) of the T = BH * ntile K tiles
+// (then, with V smoothing, BH * ntile V tiles), each smoothed by the mean of
+// its (b, h) and quantized.
 template <int D, bool kI8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    quant_k_kernel(const __grid_constant__ CUtensorMap tm_k, const QuantParams p) {
+    quant_k_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const QuantParams p) {
     extern __shared__ uint8_t smem_raw[];
     const SmemPtrs sm = smem_setup<D>(smem_raw);
     const int ntile = p.Np / kTile;
-    const long long T = static_cast<long long>(p.BH) * ntile;
+    const long long nk = static_cast<long long>(p.BH) * ntile;
+    const long long T = nk * (p.vsmooth ? 2 : 1);
     const int i0 = static_cast<int>(T * blockIdx.x / gridDim.x);
     const int i1 = static_cast<int>(T * (blockIdx.x + 1) / gridDim.x);
     const uint64_t pol = l2_policy_evict_first();
+    auto issue = [&](int s, int idx) {
+        const bool isv = idx >= nk;
+        const int ii = isv ? idx - static_cast<int>(nk) : idx;
+        ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, isv ? &tm_v : &tm_k, ii / ntile, ii % ntile,
+                      pol);
+    };
     int issued = 0;
-    // K is an input of this launch, not an output of the first one: its
+    // K and V are inputs of this launch, not outputs of the first one: their
     // loads may start before the wait below
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages && i0 + s < i1; ++s, ++issued)
-            ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, &tm_k, (i0 + s) / ntile, (i0 + s) % ntile,
-                          pol);
+        for (int s = 0; s < kStages && i0 + s < i1; ++s, ++issued) issue(s, i0 + s);
     }
     pdl_wait();
-    int cur_bh = -1;
+    int cur = -1;  // (kind, bh) whose mean is in neg_mean
     int n = 0;
     bool ok = true;
     for (; i0 + n < i1; ++n) {
         const int idx = i0 + n;
-        const int bh = idx / ntile;
-        const int tile = idx % ntile;
-        if (bh != cur_bh) {
-            // mean of K over its N tokens: chunk sums added in chunk order
-            // (fp64), one division, one rounding to fp32; the CTA holding
-            // tile 0 of this (b, h) also stores it
+        const bool isv = idx >= nk;
+        const int ii = isv ? idx - static_cast<int>(nk) : idx;
+        const int bh = ii / ntile;
+        const int tile = ii % ntile;
+        if ((isv ? p.BH : 0) + bh != cur) {
+            // mean over the N tokens: chunk sums added in chunk order (fp64),
+            // one division, one rounding to fp32; the CTA holding tile 0 of
+            // this (b, h) also stores it
+            const double *part = (isv ? p.vpart : p.part) + static_cast<size_t>(bh) * p.nchunk * D;
+            float *mean_out = isv ? p.v_mean : p.k_mean;
             for (int c = static_cast<int>(threadIdx.x); c < D; c += kThreads) {
-                const double *part = p.part + static_cast<size_t>(bh) * p.nchunk * D + c;
                 double v[kMaxChunks];
 #pragma unroll
-                for (int ch = 0; ch < kMaxChunks; ++ch) v[ch] = ch < p.nchunk ? part[static_cast<size_t>(ch) * D] : 0.0;
-                double s = 0.0;
+                for (int ch = 0; ch < kMaxChunks; ++ch)
+                    v[ch] = ch < p.nchunk ? part[static_cast<size_t>(ch) * D + c] : 0.0;
+                double sum = 0.0;
 #pragma unroll
                 for (int ch = 0; ch < kMaxChunks; ++ch)
-                    if (ch < p.nchunk) s += v[ch];
-                const float mu = __double2float_rn(s / static_cast<double>(p.N));
+                    if (ch < p.nchunk) sum += v[ch];
+                const float mu = __double2float_rn(sum / static_cast<double>(p.N));
                 sm.neg_mean[c] = -mu;
-                if (tile == 0) p.k_mean[static_cast<size_t>(bh) * D + c] = mu;
+                if (tile == 0) mean_out[static_cast<size_t>(bh) * D + c] = mu;
             }
             __syncthreads();
-            cur_bh = bh;
+            cur = (isv ? p.BH : 0) + bh;
         }
         const int s = n % kStages;
         const bool got = mbar_wait(sm.full + s, (n / kStages) & 1, sm.abort);
@@ -634,20 +665,25 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             ok = false;
             break;
         }
-        if constexpr (kI8)
-            qk_tile_i8<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean,
+        const uint8_t *st = sm.base + s * QCfg<D>::kTileBytes;
+        if constexpr (kI8) {
+            qk_tile_i8<D, true>(st, p.N, tile, sm.neg_mean,
                                 reinterpret_cast<int8_t *>(p.k_fp4) + static_cast<size_t>(bh) * p.Np * D,
                                 p.k_scale + static_cast<size_t>(bh) * (p.Np / kTile), reinterpret_cast<float *>(sm.red),
                                 p.st32 != 0);
-        else
-            qk_tile<D, true>(sm.base + s * QCfg<D>::kTileBytes, p.N, tile, sm.neg_mean, sm.lut,
-                             p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
-                             p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16), p.st32 != 0);
+        } else {
+            if (isv)
+                v_tile<D, true>(st, p.N, p.Np, tile, sm.neg_mean, sm.lut,
+                                p.vt_fp4 + static_cast<size_t>(bh) * D * (p.Np / 2),
+                                p.vt_sf + static_cast<size_t>(bh) * p.Np * 8);
+            else
+                qk_tile<D, true>(st, p.N, tile, sm.neg_mean, sm.lut, p.k_fp4 + static_cast<size_t>(bh) * p.Np * (D / 2),
+                                 p.k_sf + static_cast<size_t>(bh) * p.Np * (D / 16), p.st32 != 0);
+        }
         __syncthreads();  // stage s and neg_mean have been read by every thread
         if (threadIdx.x == 0 && i0 + n + kStages < i1) {
             fence_proxy_async_smem();
-            const int nx = i0 + n + kStages;
-            ring_issue<D>(sm.base + s * QCfg<D>::kTileBytes, sm.full + s, &tm_k, nx / ntile, nx % ntile, pol);
+            issue(s, i0 + n + kStages);
             ++issued;
         }
     }
@@ -665,14 +701,14 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
     if (e != cudaSuccess) return e;
     const int nsm = sm_count();
     const long long ntile = p.Np / kTile;
-    const long long work_a = static_cast<long long>(p.BH) * (p.Npq / kTile + ntile) +
-                             static_cast<long long>(p.BH) * p.nchunk;
+    const long long work_a = static_cast<long long>(p.BH) * (p.Npq / kTile + (p.vsmooth ? 0 : ntile)) +
+                             static_cast<long long>(p.BH) * p.nchunk * (p.vsmooth ? 2 : 1);
     const long long slots = static_cast<long long>(nsm) * kCtasPerSm;
     const int grid_a = static_cast<int>(work_a < slots ? work_a : slots);
     quant_qvk_kernel<D, kI8><<<grid_a, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const long long tiles_k = p.BH * ntile;
+    const long long tiles_k = p.BH * ntile * (p.vsmooth ? 2 : 1);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles_k < slots ? tiles_k : slots));
     cfg.blockDim = dim3(kThreads);
@@ -683,7 +719,7 @@ cudaError_t launch_d(const QuantParams &p, const CUtensorMap &tq, const CUtensor
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quant_k_kernel<D, kI8>, tk, p);
+    return cudaLaunchKernelEx(&cfg, quant_k_kernel<D, kI8>, tk, tv, p);
 }
 
 }  // namespace quant

@@ -19,6 +19,7 @@
 
 #include "attn.cuh"
 #include "attn8.cuh"
+#include "probe.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -70,6 +71,26 @@ bool make_qkv_map(CUtensorMap *m, const void *base, int d, int N, int BH) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte range [p, p + n) of a buffer.
+struct Range {
+    uintptr_t lo, hi;
+};
+Range range_of(const void *p, int64_t n) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + static_cast<uintptr_t>(n)};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// True if any written range overlaps any input range.  The quantizer's
+// second launch loads K before it waits for the first launch, so an output
+// that aliases an input would race with those loads.
+bool any_overlap(const Range *in, int nin, const Range *out, int nout) {
+    for (int i = 0; i < nin; ++i)
+        for (int o = 0; o < nout; ++o)
+            if (overlap(in[i], out[o])) return true;
+    return false;
+}
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 int check_shape(int B, int H, int N, int d) {
@@ -132,15 +153,31 @@ extern "C" {
 
 const char *sa3_version(void) { return "libsa3 0.1.0 (sm_100a)"; }
 
-int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, int H, int Nq, int Nkv, int d,
-                          const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes,
-                          struct CUstream_st *stream) {
+int sa3_quantize_qkv_ex(const void *q, const void *k, const void *v, int B, int H, int Nq, int Nkv, int d,
+                        unsigned int flags, const sa3_qkv_fp4 *out, float *v_mean, void *workspace,
+                        size_t workspace_bytes, struct CUstream_st *stream) {
     int rc = check_shape(B, H, Nq, d);
     if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
+    if ((flags & ~static_cast<unsigned int>(SA3_V_SMOOTH)) != 0) return SA3_ERR_INVALID_ARG;
+    const bool vsmooth = (flags & SA3_V_SMOOTH) != 0;
     if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
     if ((rc = check_qkv(out)) != SA3_OK) return rc;
-    const int64_t need = sa3_quant_workspace_bytes(B, H, Nkv, d);
+    if (vsmooth && (!v_mean || !aligned16(v_mean))) return SA3_ERR_INVALID_ARG;
+    const int64_t need = sa3_quant_workspace_bytes_ex(B, H, Nkv, d, flags);
     if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
+    {
+        const Range in[3] = {range_of(q, int64_t(B) * H * Nq * d * 2), range_of(k, int64_t(B) * H * Nkv * d * 2),
+                             range_of(v, int64_t(B) * H * Nkv * d * 2)};
+        const Range wr[9] = {range_of(out->q_fp4, sa3_qk_fp4_bytes(B, H, Nq, d)),
+                             range_of(out->q_sf, sa3_qk_sf_bytes(B, H, Nq, d)),
+                             range_of(out->k_fp4, sa3_qk_fp4_bytes(B, H, Nkv, d)),
+                             range_of(out->k_sf, sa3_qk_sf_bytes(B, H, Nkv, d)),
+                             range_of(out->vt_fp4, sa3_vt_fp4_bytes(B, H, Nkv, d)),
+                             range_of(out->vt_sf, sa3_vt_sf_bytes(B, H, Nkv, d)),
+                             range_of(out->k_mean, sa3_kmean_bytes(B, H, d)), range_of(workspace, need),
+                             range_of(v_mean, vsmooth ? sa3_kmean_bytes(B, H, d) : 0)};
+        if (any_overlap(in, 3, wr, 9)) return SA3_ERR_INVALID_ARG;
+    }
     sa3::QuantParams p = {};
     p.q_fp4 = static_cast<uint8_t *>(out->q_fp4);
     p.q_sf = static_cast<uint8_t *>(out->q_sf);
@@ -158,12 +195,21 @@ int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, in
     p.chunk = static_cast<int>(sa3_kmean_chunk(Nkv));
     p.nchunk = static_cast<int>(sa3_kmean_nchunk(Nkv));
     p.st32 = aligned32(p.q_fp4) && aligned32(p.k_fp4);
+    p.vsmooth = vsmooth ? 1 : 0;
+    p.v_mean = v_mean;
+    p.vpart = p.part + static_cast<size_t>(p.BH) * p.nchunk * d;
     CUtensorMap tq, tk, tv;
     if (!make_qkv_map(&tq, q, d, Nq, p.BH) || !make_qkv_map(&tk, k, d, Nkv, p.BH) ||
         !make_qkv_map(&tv, v, d, Nkv, p.BH))
         return SA3_ERR_CUDA;
     return sa3::launch_quant(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK
                                                                                                         : SA3_ERR_CUDA;
+}
+
+int sa3_quantize_qkv_lens(const void *q, const void *k, const void *v, int B, int H, int Nq, int Nkv, int d,
+                          const sa3_qkv_fp4 *out, void *workspace, size_t workspace_bytes,
+                          struct CUstream_st *stream) {
+    return sa3_quantize_qkv_ex(q, k, v, B, H, Nq, Nkv, d, 0u, out, nullptr, workspace, workspace_bytes, stream);
 }
 
 int sa3_quantize_qkv_i8(const void *q, const void *k, const void *v, int B, int H, int Nq, int Nkv, int d,
@@ -178,6 +224,17 @@ int sa3_quantize_qkv_i8(const void *q, const void *k, const void *v, int B, int 
         return SA3_ERR_INVALID_ARG;
     const int64_t need = sa3_quant_workspace_bytes(B, H, Nkv, d);
     if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
+    {
+        const Range in[3] = {range_of(q, int64_t(B) * H * Nq * d * 2), range_of(k, int64_t(B) * H * Nkv * d * 2),
+                             range_of(v, int64_t(B) * H * Nkv * d * 2)};
+        const Range wr[7] = {range_of(out->q_i8, sa3_i8_bytes(B, H, Nq, d)),
+                             range_of(out->q_scale, sa3_i8_scale_bytes(B, H, Nq)),
+                             range_of(out->k_i8, sa3_i8_bytes(B, H, Nkv, d)),
+                             range_of(out->k_scale, sa3_i8_scale_bytes(B, H, Nkv)),
+                             range_of(out->vt_f16, sa3_vt_f16_bytes(B, H, Nkv, d)),
+                             range_of(out->k_mean, sa3_kmean_bytes(B, H, d)), range_of(workspace, need)};
+        if (any_overlap(in, 3, wr, 7)) return SA3_ERR_INVALID_ARG;
+    }
     sa3::QuantParams p = {};
     p.q_fp4 = static_cast<uint8_t *>(out->q_i8);
     p.k_fp4 = static_cast<uint8_t *>(out->k_i8);
@@ -223,13 +280,14 @@ int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B,
     return sa3_quantize_qkv(q, k, v, B, H, N, d, out, scratch, SA3_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
-                      unsigned int flags, void *out, struct CUstream_st *stream) {
+int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean, int B, int H, int Nq, int Nkv, int d, int causal,
+                    float sm_scale, unsigned int flags, void *out, struct CUstream_st *stream) {
     int rc = check_shape(B, H, Nq, d);
     if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
     if ((rc = check_qkv(in)) != SA3_OK) return rc;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
-    if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL)) != 0) return SA3_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL | SA3_V_SMOOTH)) != 0) return SA3_ERR_INVALID_ARG;
+    if ((flags & SA3_V_SMOOTH) && (!v_mean || !aligned16(v_mean))) return SA3_ERR_INVALID_ARG;
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
     const int BH = B * H;
@@ -241,11 +299,12 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
         !make_map(&tk, in->k_fp4, d / 2, static_cast<uint64_t>(BH) * Np, d / 2, 128, qk_sw) ||
         !make_map(&tv, in->vt_fp4, Np / 2, static_cast<uint64_t>(BH) * d, 64, d, CU_TENSOR_MAP_SWIZZLE_64B))
         return SA3_ERR_CUDA;
-    sa3::AttnParams p;
+    sa3::AttnParams p = {};
     p.q_sf = static_cast<const uint8_t *>(in->q_sf);
     p.k_sf = static_cast<const uint8_t *>(in->k_sf);
     p.vt_sf = static_cast<const uint8_t *>(in->vt_sf);
     p.out = static_cast<__nv_bfloat16 *>(out);
+    p.v_mean = (flags & SA3_V_SMOOTH) ? v_mean : nullptr;
     p.BH = BH;
     p.N = Nkv;
     p.Np = Np;
@@ -257,6 +316,12 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
     return sa3::launch_attn(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA3_OK
                : SA3_ERR_CUDA;
+}
+
+int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                      unsigned int flags, void *out, struct CUstream_st *stream) {
+    if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL)) != 0) return SA3_ERR_INVALID_ARG;
+    return sa3_attn_fwd_ex(in, nullptr, B, H, Nq, Nkv, d, causal, sm_scale, flags, out, stream);
 }
 
 int sa3_attn_fwd_i8_lse(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
@@ -305,6 +370,16 @@ int sa3_attn_fwd_i8(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, 
 int sa3_attn_fwd(const sa3_qkv_fp4 *in, int B, int H, int N, int d, int causal, float sm_scale, void *out,
                  struct CUstream_st *stream) {
     return sa3_attn_fwd_lens(in, B, H, N, N, d, causal, sm_scale, 0u, out, stream);
+}
+
+int sa3_probe_fp4_mma(int ctas, int n, int iters, float *out, struct CUstream_st *stream) {
+    if (ctas < 1 || ctas > 65535 || iters < 1 || iters > (1 << 18) || !out || (n != 128 && n != 256) ||
+        (reinterpret_cast<uintptr_t>(out) & 3u))
+        return SA3_ERR_INVALID_ARG;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = n == 128 ? sa3::probe::launch<128>(ctas, iters, out, s)
+                                   : sa3::probe::launch<256>(ctas, iters, out, s);
+    return e == cudaSuccess ? SA3_OK : SA3_ERR_CUDA;
 }
 
 int sa3_selftest_wait_timeout(unsigned int limit_us, struct CUstream_st *stream) {

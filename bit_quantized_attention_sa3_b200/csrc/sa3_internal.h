@@ -22,6 +22,9 @@ struct QuantParams {
     float *q_scale;  // 8-bit variant: one fp32 scale per 128-token tile of Q
     float *k_scale;  // ... and of K (codes then go to q_fp4 / k_fp4 as int8, V to vt_fp4 as fp16)
     double *part;    // [BH][nchunk][d] scratch: fp64 column sums of K per chunk
+    double *vpart;   // ... and of V (V smoothing only)
+    float *v_mean;   // V smoothing: fp32 [BH][d] mean of V (else unused)
+    int vsmooth;     // 1: V is smoothed like K (its tiles move to the second launch)
     int BH;
     int N;       // K and V tokens
     int Np;      // N rounded up to 128
@@ -39,6 +42,7 @@ struct AttnParams {
     const float *q_scale;  // 8-bit variant: fp32 scale per 128-token tile of Q
     const float *k_scale;  // ... and of K
     __nv_bfloat16 *out;
+    const float *v_mean;  // FP4, V smoothing: fp32 [BH][d] mean of V added to every output row, or null
     float *lse;        // 8-bit variant: per-row log-sum-exp (natural log), or null
     int BH;
     int N;             // key / value tokens
@@ -49,8 +53,9 @@ struct AttnParams {
     float scale_log2;  // fp32(sm_scale * log2 e)
     float p_pre_log2;  // 0, or 11 for two-level P (P scaled by 2^11 before microscaling;
                        // selects the kernel instance, whose exponent is fixed)
-    int npairs;        // Q-tile pairs per head (set by the launcher)
-    int pair_units;    // work units that are pairs; the rest are single tiles
+    int npairs;        // 8-bit kernel: Q-tile pairs per head (set by the launcher)
+    int pair_units;    // 8-bit kernel: work units that are pairs; the rest are single tiles
+    int hg;            // FP4 kernel: heads per group of its persistent work list (set by the launcher)
 };
 
 // Host: raise Kernel's dynamic shared memory limit once per device (the

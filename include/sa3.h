@@ -34,12 +34,16 @@
  *     attributes, once.  Make it outside stream capture.  After it, the
  *     calls only enqueue kernels, with no allocation, synchronization or
  *     attribute call, so they can be recorded into a CUDA graph (stream
- *     capture) and replayed with new inputs in the same buffers.
+ *     capture) and replayed with new inputs in the same buffers;
+ *   - the quantizer's inputs (q, k, v) must not share bytes with any of its
+ *     outputs or its workspace: its second kernel starts loading K while
+ *     the first may still be writing.  Such a call is rejected.
  *
  * Error behaviour: arguments are checked before any launch; a bad argument
  * returns SA3_ERR_INVALID_ARG (null pointer, misalignment, non-positive
- * size, workspace too small) or SA3_ERR_UNSUPPORTED (d not 64/128, size
- * limits) and enqueues nothing.  A failed launch returns SA3_ERR_CUDA.
+ * size, workspace too small, an output overlapping an input) or
+ * SA3_ERR_UNSUPPORTED (d not 64/128, size limits) and enqueues nothing.
+ * A failed launch returns SA3_ERR_CUDA.
  * Device-side waits are bounded; if one gives up, the kernel records
  * SA3_ERR_TIMEOUT in a device status word, releases what it holds and
  * returns; sa3_device_status() reports it.
@@ -212,6 +216,41 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
                       struct CUstream_st *stream);
 
 /*
+ * sa3_quantize_qkv_ex, sa3_attn_fwd_ex -- the _lens calls with option flags.
+ *
+ * SA3_V_SMOOTH: V is smoothed like K.  The quantizer also forms the mean of
+ *   V over its Nkv tokens (fp64 sum, fp64 divide, one rounding to fp32, as
+ *   for K), writes it to v_mean (fp32 [B][H][d], device, 16-byte aligned,
+ *   caller-owned) and quantizes V_s = fp32(V) - mean (one fp32 subtraction;
+ *   padding tokens stay 0) instead of V.  Attention, given the same v_mean,
+ *   adds it back after O / l:  out = bf16(O / l + mean), in fp32 (a row that
+ *   sees no key still outputs 0).  Softmax rows sum to 1, so this leaves
+ *   attention unchanged in exact arithmetic -- the argument the SageAttention
+ *   summary ("Approach") gives for K, applied to V's per-channel mean -- and
+ *   it helps when V has a large per-channel offset.  The pages do not
+ *   describe it: an accuracy option, off by default.  The quantizer's
+ *   workspace doubles (V's partial sums): sa3_quant_workspace_bytes_ex.
+ *   V smoothing needs V's mean before V can be quantized, so V is read
+ *   twice (once for the sums, once to quantize).
+ * SA3_P_TWO_LEVEL (attention only): as in sa3_attn_fwd_lens.
+ *
+ * v_mean is ignored (may be NULL) without SA3_V_SMOOTH.  Any other flag bit:
+ * SA3_ERR_INVALID_ARG.  Everything else as in the _lens calls, which are
+ * these with flags 0 (quantizer) or flags without SA3_V_SMOOTH (attention).
+ */
+#define SA3_V_SMOOTH 2u
+static inline int64_t sa3_quant_workspace_bytes_ex(int64_t B, int64_t H, int64_t N, int64_t d, unsigned int flags)
+{ return sa3_quant_workspace_bytes(B, H, N, d) * ((flags & SA3_V_SMOOTH) ? 2 : 1); }
+int sa3_quantize_qkv_ex(const void *q, const void *k, const void *v,
+                        int B, int H, int Nq, int Nkv, int d, unsigned int flags,
+                        const sa3_qkv_fp4 *out, float *v_mean,
+                        void *workspace, size_t workspace_bytes,
+                        struct CUstream_st *stream);
+int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean,
+                    int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
+                    unsigned int flags, void *out, struct CUstream_st *stream);
+
+/*
  * 8-bit variant ("SageAttention: Accurate 8-Bit Attention for Plug-and-play
  * Inference Acceleration", summary, "Approach"): Q and K quantized to INT8
  * with per-block scales after K smoothing, P and V kept in FP16.  Blocks are
@@ -295,8 +334,11 @@ int sa3_attn_fwd_i8_lse(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int
  * It calls no allocation routine.
  *
  * The first call on a device looks up that device's copy of the array
- * (cudaGetSymbolAddress, with the device current); make that first call
- * outside any stream capture.  All calls share the one array: two calls
+ * (cudaGetSymbolAddress, with the device current) and keeps the address
+ * for the life of the process; make that first call outside any stream
+ * capture.  The address belongs to the device's primary context, the one
+ * the CUDA runtime and PyTorch use: call this from that context only, and
+ * not after cudaDeviceReset (the kept address is then stale).  All calls share the one array: two calls
  * whose kernels overlap on the GPU (different streams without ordering)
  * race on it and give undefined results.  Nothing in the array needs to
  * start at zero -- every call rewrites all the scratch it reads -- and it
@@ -326,6 +368,23 @@ int sa3_device_status(struct CUstream_st *stream);
  * No counterpart in the method; for tests of failure detection.
  */
 int sa3_selftest_wait_timeout(unsigned int limit_us, struct CUstream_st *stream);
+
+/*
+ * sa3_probe_fp4_mma -- measures the block-scaled FP4 tensor-core rate that
+ * bounds sa3_attn_fwd.  No counterpart in the method: a measurement aid for
+ * the attention roofline.  Enqueues `ctas` CTAs (one per SM when ctas is
+ * the SM count; each claims enough shared memory to be alone on its SM),
+ * each issuing `iters` (1 .. 2^18) tcgen05.mma.kind::mxf4nvf4 block-scaled
+ * MMAs of M = 128, N = n (128 or 256), K = 64 from shared memory into one
+ * TMEM accumulator: 2 * 128 * n * 64 operations each.  All codes are E2M1
+ * 1.0 and all scales E4M3 1.0, so every accumulator element ends at
+ * exactly 64 * iters.  out: device fp32 [2 * ctas], 4-byte aligned; CTA c
+ * writes the smallest element of accumulator column 0 to out[2c] and the
+ * largest of column n-1 to out[2c+1] (both 64 * iters when the tensor core
+ * did the work).  The caller times the launch (CUDA events on `stream`).
+ * Bad arguments: SA3_ERR_INVALID_ARG; launch failure: SA3_ERR_CUDA.
+ */
+int sa3_probe_fp4_mma(int ctas, int n, int iters, float *out, struct CUstream_st *stream);
 
 /* Library version string, e.g. "libsa3 0.1.0 (sm_100a)". Host memory,
  * static, never freed. */

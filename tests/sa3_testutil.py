@@ -93,3 +93,75 @@ def sample_units(B: int, H: int, N: int, seed: int = 0, per_bh: int = 2, bh_list
                                                       replace=False))
         units += [(bh, qb) for qb in sorted(blocks)]
     return units
+
+
+# ------------------------------------------------- end-to-end parity chain
+def gpu_canonical(qz, B: int, H: int, Nq: int, Nkv: int, d: int) -> dict:
+    """The GPU's quantized operands in the oracle's canonical layout."""
+    Npq = (Nq + 127) // 128 * 128
+    Np = (Nkv + 127) // 128 * 128
+    g = {f: getattr(qz, f).cpu().numpy() for f in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean")}
+    return dict(q_codes=g["q_fp4"].reshape(B, H, Npq, d // 2), k_codes=g["k_fp4"].reshape(B, H, Np, d // 2),
+                vt_codes=g["vt_fp4"].reshape(B, H, d, Np // 2), k_mean=g["k_mean"].reshape(B, H, d),
+                q_sf=qk_sf_to_canonical(g["q_sf"], B, H, Npq, d), k_sf=qk_sf_to_canonical(g["k_sf"], B, H, Np, d),
+                vt_sf=vt_sf_to_canonical(g["vt_sf"], B, H, Np, d), vt_sf_pad=vt_sf_padding(g["vt_sf"], B, H, Np, d))
+
+
+def heads_of(t: torch.Tensor, bh_list) -> torch.Tensor:
+    """Heads bh_list of a [B,H,N,d] tensor, stacked as [1, len, N, d]."""
+    B, H, N, d = t.shape
+    return t.reshape(B * H, N, d)[list(bh_list)].reshape(1, len(bh_list), N, d).contiguous()
+
+
+def oracle_quantize_heads(oracle, q, k, v, bh_list, **kw) -> dict:
+    """The oracle's own quantization of heads bh_list (one head's result does
+    not depend on the others), as a B=1, H=len(bh_list) operand set."""
+    return oracle.quantize_qkv(heads_of(q, bh_list), heads_of(k, bh_list), heads_of(v, bh_list), **kw)
+
+
+def assert_quantized_equal(gpu: dict, ref: dict, bh_list) -> None:
+    """Codes, scales and the K mean of the GPU (canonical, all heads) equal
+    the oracle's (heads bh_list only), bit for bit."""
+    idx = list(bh_list)
+    for f in ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf"):
+        g = gpu[f].reshape((-1,) + gpu[f].shape[2:])[idx]
+        r = ref[f].reshape((-1,) + ref[f].shape[2:])
+        if not np.array_equal(g, r):
+            bad = np.argwhere(g != r)
+            raise AssertionError(f"{f}: {len(bad)} bytes differ from the oracle's, first (head, ...) "
+                                 f"{[[idx[b[0]]] + b[1:].tolist() for b in bad[:4]]}")
+    gm = gpu["k_mean"].reshape(-1, gpu["k_mean"].shape[-1])[idx]
+    rm = ref["k_mean"].reshape(-1, ref["k_mean"].shape[-1])
+    assert np.array_equal(gm.view(np.uint32), rm.view(np.uint32)), "k_mean differs from the oracle's"
+    if "vt_sf_pad" in gpu:
+        assert not gpu["vt_sf_pad"].any(), "padding channels of the V^T scale atoms are not 0"
+
+
+def blockwise_rel_l2(got: np.ndarray, ref: np.ndarray, blocks, tol: float, live=None, label: str = "") -> float:
+    """rel-L2 of got against ref for every (head, Q block) in ``blocks``
+    (got, ref: [heads, Nq, d] float arrays; blocks: (head index, q_block)
+    pairs; live: optional [Nq] mask of rows that see a key).  Fails on the
+    first block above ``tol``; prints the worst block and the worst single
+    element.  Returns the worst block's error."""
+    Nq = got.shape[1]
+    worst, where = 0.0, None
+    for h, qb in blocks:
+        rows = np.arange(qb * 128, min(Nq, qb * 128 + 128))
+        if live is not None:
+            rows = rows[live[rows]]
+        if rows.size == 0:
+            continue
+        g = got[h, rows].astype(np.float64)
+        r = ref[h, rows].astype(np.float64)
+        nr = np.linalg.norm(r)
+        err = np.linalg.norm(g - r) / nr if nr > 0 else np.linalg.norm(g)
+        if err > worst:
+            worst, where = err, (h, qb)
+    dif = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    if live is not None:
+        dif = dif[:, live]
+    e = np.unravel_index(np.argmax(dif), dif.shape) if dif.size else ()
+    print(f"{label} worst block rel-L2 {worst:.3e} at (head, q_block) {where}; "
+          f"worst element |diff| {dif.max() if dif.size else 0.0:.3e} at {tuple(int(x) for x in e)}")
+    assert worst <= tol, f"{label} block {where}: rel-L2 {worst:.3e} > {tol}"
+    return worst

@@ -26,8 +26,9 @@ def lib():
 
 
 def test_header_declares_the_boundary():
-    assert _declared() == ["sa3_attn_fwd", "sa3_attn_fwd_i8", "sa3_attn_fwd_i8_lse", "sa3_attn_fwd_lens", "sa3_device_status",
-                           "sa3_quantize_qkv", "sa3_quantize_qkv_i8", "sa3_quantize_qkv_lens",
+    assert _declared() == ["sa3_attn_fwd", "sa3_attn_fwd_ex", "sa3_attn_fwd_i8", "sa3_attn_fwd_i8_lse",
+                           "sa3_attn_fwd_lens", "sa3_device_status", "sa3_probe_fp4_mma", "sa3_quantize_qkv",
+                           "sa3_quantize_qkv_ex", "sa3_quantize_qkv_i8", "sa3_quantize_qkv_lens",
                            "sa3_quantize_qkv_noalloc", "sa3_selftest_wait_timeout", "sa3_version"]
 
 
@@ -61,6 +62,12 @@ def test_argument_checks_need_no_gpu(lib):
     lib.sa3_selftest_wait_timeout.restype = I
     lib.sa3_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     assert lib.sa3_selftest_wait_timeout(0, None) == 1
+    lib.sa3_probe_fp4_mma.restype = I
+    lib.sa3_probe_fp4_mma.argtypes = [I, I, I, P, P]
+    assert lib.sa3_probe_fp4_mma(148, 192, 16, 16, None) == 1     # n must be 128 or 256
+    assert lib.sa3_probe_fp4_mma(148, 128, 0, 16, None) == 1      # iters >= 1
+    assert lib.sa3_probe_fp4_mma(148, 128, 1 << 19, 16, None) == 1
+    assert lib.sa3_probe_fp4_mma(148, 128, 16, None, None) == 1
     # separate query / key lengths: each is checked
     lib.sa3_quantize_qkv_lens.restype = I
     lib.sa3_quantize_qkv_lens.argtypes = [P, P, P, I, I, I, I, I, P, P, ctypes.c_size_t, P]

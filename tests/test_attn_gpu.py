@@ -1,9 +1,16 @@
-"""sa3_attn_fwd on the GPU against the CPU oracle.
+"""sa3_attn_fwd on the GPU against the CPU oracle, end to end.
 
-Bar: output rel-L2 <= 2e-3 against the oracle on the same quantized
-operands (the GPU takes its exponentials with ex2.approx and accumulates in
-the tensor core, so P codes may flip at rounding boundaries; the oracle
-uses exp2f and fp64 sums).  The GPU is also checked against fp64 exact
+Chain: the oracle quantizes the same bf16 inputs itself (only the heads
+under test), the GPU's codes, scales and K mean must equal its own bit for
+bit, and the oracle then attends on ITS OWN quantized operands.  So a
+quantizer fault shared by both sides cannot hide behind the attention
+comparison.
+
+Bar: output rel-L2 <= 2e-3 against the oracle in every (head, 128-row Q
+block) compared (the GPU takes its exponentials with ex2.approx and
+accumulates in the tensor core, so P codes may flip at rounding
+boundaries; the oracle uses exp2f and fp64 sums).  The worst block and the
+worst element are printed.  The GPU is also checked against fp64 exact
 attention of the bf16 inputs: its cosine must be within 1e-3 of the
 oracle's own cosine (the method's accuracy, not a kernel property).
 
@@ -16,44 +23,51 @@ import torch
 
 import oracle
 import sa3_inputs
-from sa3_testutil import bits_to_f32, cosine, qk_sf_to_canonical, rel_l2, sample_units, vt_sf_to_canonical
+from sa3_testutil import (assert_quantized_equal, bits_to_f32, blockwise_rel_l2, cosine, gpu_canonical, heads_of,
+                          oracle_quantize_heads, sample_units)
 
 sa3 = pytest.importorskip("bit_quantized_attention_sa3_b200")
 
 TOL = 2e-3
 
 
-def _canonical(qz, B, H, N, d):
-    Np = sa3.padded_len(N)
-    return dict(q_codes=qz.q_fp4.cpu().numpy(), k_codes=qz.k_fp4.cpu().numpy(),
-                vt_codes=qz.vt_fp4.cpu().numpy(),
-                q_sf=qk_sf_to_canonical(qz.q_sf.cpu().numpy(), B, H, Np, d),
-                k_sf=qk_sf_to_canonical(qz.k_sf.cpu().numpy(), B, H, Np, d),
-                vt_sf=vt_sf_to_canonical(qz.vt_sf.cpu().numpy(), B, H, Np, d))
+def _chain(q, k, v, qz, out, causal, units=None, bh_list=None, sm_scale=None, label="", two=False):
+    """Oracle chain on heads bh_list (default all): quantization bit-exact,
+    then per-block rel-L2 of out against the oracle's attention on its own
+    operands.  Returns (worst block rel-L2, cosine gpu vs exact, cosine
+    oracle vs exact) over the compared rows."""
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    heads = list(range(B * H)) if bh_list is None else list(bh_list)
+    pos = {bh: i for i, bh in enumerate(heads)}
+    ref_q = oracle_quantize_heads(oracle, q, k, v, heads)
+    assert_quantized_equal(gpu_canonical(qz, B, H, Nq, Nkv, d), ref_q, heads)
+    nqb = (Nq + 127) // 128
+    if units is None:
+        units = [(bh, qb) for bh in heads for qb in range(nqb)]
+    sub = [(pos[bh], qb) for bh, qb in units]
+    ref = bits_to_f32(oracle.attn_fwd(ref_q, Nq, causal, units=sub, sm_scale=sm_scale, p_two_level=two))[0]
+    ex = oracle.attn_exact(heads_of(q, heads), heads_of(k, heads), heads_of(v, heads), causal, units=sub,
+                           sm_scale=sm_scale)[0]
+    got = out.float().cpu().numpy().reshape(B * H, Nq, d)[heads]
+    assert np.isfinite(got).all()
+    live = (np.arange(Nq) + (Nkv - Nq) >= 0) if causal else None
+    worst = blockwise_rel_l2(got, ref, sub, TOL, live=live, label=label)
+    mask = np.zeros((len(heads), Nq), bool)
+    for h, qb in sub:
+        mask[h, qb * 128: min(Nq, qb * 128 + 128)] = True
+    if live is not None:
+        mask &= live[None, :]
+    return worst, cosine(got[mask], ex[mask]), cosine(ref[mask], ex[mask])
 
 
-def _run(name, over, causal, units=None):
+def _run(name, over, causal, units=None, bh_list=None):
     q, k, v = sa3_inputs.make_qkv(name, shape_override=over)
-    B, H, N, d = q.shape
     qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
     out = sa3.attn_fwd(qz, causal=causal)
     torch.cuda.synchronize()
     assert sa3.device_status() == sa3.SA3_OK
-    got = out.float().cpu().numpy()
-    assert np.isfinite(got).all()
-    canon = _canonical(qz, B, H, N, d)
-    ref = bits_to_f32(oracle.attn_fwd(canon, N, causal, units=units))
-    ex = oracle.attn_exact(q, k, v, causal, units=units)
-    if units is None:
-        mask = np.ones((B * H, N), bool)
-    else:
-        mask = np.zeros((B * H, N), bool)
-        for bh, qb in units:
-            mask[bh, qb * 128: min(N, qb * 128 + 128)] = True
-    g = got.reshape(B * H, N, d)[mask]
-    r = ref.reshape(B * H, N, d)[mask]
-    e = ex.reshape(B * H, N, d)[mask]
-    return rel_l2(g, r), cosine(g, e), cosine(r, e)
+    return _chain(q, k, v, qz, out, causal, units=units, bh_list=bh_list, label=name)
 
 
 SMALL = [
@@ -101,38 +115,53 @@ def test_attn_matches_oracle_full_size_sampled(case):
         rng = np.random.default_rng(2)
         bh_list = sorted({0, w.B * w.H - 1} | set(int(x) for x in rng.choice(w.B * w.H, 14, replace=False)))
     units = sample_units(w.B, w.H, w.N, seed=3, per_bh=2, bh_list=bh_list)
-    err, cos_gpu, cos_oracle = _run(name, None, causal, units=units)
-    print(f"{name}: rel-L2 vs oracle {err:.3e}, cosine vs exact gpu {cos_gpu:.5f} oracle {cos_oracle:.5f}")
+    heads = sorted({bh for bh, _ in units})
+    err, cos_gpu, cos_oracle = _run(name, None, causal, units=units, bh_list=heads)
+    print(f"{name}: worst block rel-L2 vs oracle {err:.3e}, cosine vs exact gpu {cos_gpu:.5f} "
+          f"oracle {cos_oracle:.5f}")
     assert err <= TOL
     assert cos_gpu >= cos_oracle - 1e-3
 
 
 @pytest.mark.gpu
 def test_attn_sm_scale_and_repeatability():
-    q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 384})]
-    B, H, N, d = q.shape
-    qz = sa3.quantize_qkv(q, k, v)
+    q, k, v = sa3_inputs.make_qkv("tiny_b1h2n256d64", shape_override={"N": 384})
+    qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
     a = sa3.attn_fwd(qz, causal=False, sm_scale=0.05)
     b = sa3.attn_fwd(qz, causal=False, sm_scale=0.05)
+    c = sa3.attn_fwd(qz, causal=False)
+    d0 = sa3.attn_fwd(qz, causal=False, sm_scale=1.0 / 8.0)  # 1/sqrt(64): the library's default
     torch.cuda.synchronize()
     assert torch.equal(a, b)
-    canon = _canonical(qz, B, H, N, d)
-    ref = bits_to_f32(oracle.attn_fwd(canon, N, False, sm_scale=0.05))
-    assert rel_l2(a.float().cpu().numpy(), ref) <= TOL
+    assert torch.equal(c, d0)
+    _chain(q, k, v, qz, a, False, sm_scale=0.05, label="sm_scale 0.05")
 
 
 @pytest.mark.gpu
 def test_attn_rejects_bad_arguments():
+    import ctypes
     q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64")]
+    B, H, N, d = q.shape
     qz = sa3.quantize_qkv(q, k, v)
-    bad = sa3.QuantizedQKV(**{**qz.__dict__, "d": 80})
-    with pytest.raises(sa3.Sa3Error) as e:
-        sa3.attn_fwd(bad)
-    assert e.value.code == sa3.SA3_ERR_UNSUPPORTED
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream().cuda_stream
+    # d = 80: the library does not support it (the binding's size check
+    # fails first, since the buffers were sized for d = 64)
+    rc = sa3.lib().sa3_attn_fwd(ctypes.byref(qz.struct()), B, H, N, 80, 0, 0.0, out.data_ptr(), stream)
+    assert rc == sa3.SA3_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        sa3.attn_fwd(sa3.QuantizedQKV(**{**qz.__dict__, "d": 80}))
+    # an output buffer that is not 16-byte aligned
     mis = torch.empty(q.numel() + 8, dtype=torch.bfloat16, device="cuda")[1:1 + q.numel()].view(q.shape)
     with pytest.raises(sa3.Sa3Error) as e:
         sa3.attn_fwd(qz, out=mis)
     assert e.value.code == sa3.SA3_ERR_INVALID_ARG
+    # wrong shape, dtype or device of out: refused before any launch
+    for bad in (torch.empty((B, H, N - 1, d), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((B, H, N, d), dtype=torch.float16, device="cuda"),
+                torch.empty((B, H, N, d), dtype=torch.bfloat16)):
+        with pytest.raises(ValueError):
+            sa3.attn_fwd(qz, out=bad)
 
 
 @pytest.mark.gpu
@@ -150,21 +179,30 @@ def test_attn_tail_wave_single_tile_units(causal):
 @pytest.mark.gpu
 def test_causal_row0_matches_oracle_exactly():
     """Row 0 sees key 0 only (P = [1, 0, ...], one code and scale decision):
-    the GPU must give the oracle's bf16(1.03125 * v^_0) to within one bf16
-    ulp, on inputs whose row-0 logits reach far below zero.  (The GPU folds
-    log2(1/s) into the exp2 argument, -m' + log2(1/s) rounded at the size of
-    m', so with logits in the thousands P carries ~1e-4 relative error and
-    some outputs land one ulp away.)"""
+    the GPU must give the oracle's bf16(1.03125 * v^_0), on inputs whose
+    row-0 logits reach the hundreds (outlier channels), where the exponent
+    argument has to be formed in the oracle's order of roundings."""
     q, k, v = sa3_inputs.make_qkv("prefill_b4h32n8192d128_causal", shape_override={"B": 1, "H": 32, "N": 1024})
     B, H, N, d = q.shape
     qz = sa3.quantize_qkv(q.cuda(), k.cuda(), v.cuda())
     out = sa3.attn_fwd(qz, causal=True)
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
-    ref = oracle.attn_fwd(_canonical(qz, B, H, N, d), N, True, units=[(bh, 0) for bh in range(B * H)])
+    r = oracle.quantize_qkv(q, k, v)
+    assert_quantized_equal(gpu_canonical(qz, B, H, N, N, d), r, range(B * H))
+    ref = oracle.attn_fwd(r, N, True, units=[(bh, 0) for bh in range(B * H)])
     got = out[:, :, 0].float().cpu().numpy()
     want = bits_to_f32(ref[:, :, 0])
+    # one bf16 ulp at most: the GPU's row sum is sum_b s_b * sum(P / s_b)
+    # with the hardware exp2, so l may sit one fp32 ulp off 1 and decide a
+    # bf16 tie of 1.03125 * v^_0 the other way; every other output is equal
     assert np.all(np.abs(got - want) <= 2.0 ** -7 * np.abs(want))
+    same = float(np.mean(got == want))
+    print(f"row 0: {same:.4f} of outputs identical to the oracle's")
+    # about a quarter of the values 1.03125 * v^ are exact bf16 ties, decided
+    # by the last fp32 bit of l; warps whose rows all have |m'| < 32 form l
+    # through the folded exponent, which can move that bit
+    assert same >= 0.85
 
 
 @pytest.mark.gpu
@@ -181,20 +219,9 @@ def test_long_sequence_131072_tokens(causal):
     out = sa3.attn_fwd(qz, causal=causal)
     torch.cuda.synchronize()
     assert sa3.device_status() == sa3.SA3_OK
-    canon = _canonical(qz, B, H, N, d)
-    if not causal:  # the quantized operands do not depend on the mask: compare once
-        r = oracle.quantize_qkv(q, k, v)
-        for f in ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf"):
-            assert np.array_equal(canon[f], r[f]), f
-        assert np.array_equal(qz.k_mean.cpu().numpy().view(np.uint32), r["k_mean"].view(np.uint32))
     nqb = N // 128
     units = [(bh, qb) for bh in range(B * H) for qb in (0, nqb - 1, 517)]
-    ref = bits_to_f32(oracle.attn_fwd(canon, N, causal, units=units)).reshape(B * H, N, d)
-    got = out.float().cpu().numpy().reshape(B * H, N, d)
-    assert np.isfinite(got).all()
-    for bh, qb in units:
-        rows = slice(qb * 128, qb * 128 + 128)
-        assert rel_l2(got[bh, rows], ref[bh, rows]) <= TOL, (bh, qb)
+    _chain(q, k, v, qz, out, causal, units=units, label=f"N=131072 causal={causal}")
 
 
 @pytest.mark.gpu
@@ -210,12 +237,4 @@ def test_many_heads_beyond_65535(causal):
     out = sa3.attn_fwd(qz, causal=causal)
     torch.cuda.synchronize()
     assert sa3.device_status() == sa3.SA3_OK
-    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
-    codes = qz.k_fp4.cpu().numpy()
-    for bh in (0, 65535, 65536, B * H - 1):
-        b, h = divmod(bh, H)
-        sl = slice(b, b + 1), slice(h, h + 1)
-        r = oracle.quantize_qkv(q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous())
-        assert np.array_equal(codes[b, h], r["k_codes"][0, 0]), bh
-        ref = bits_to_f32(oracle.attn_fwd(r, N, causal))[0, 0]
-        assert rel_l2(bits_to_f32(got[b, h]), ref) <= TOL, bh
+    _chain(q, k, v, qz, out, causal, bh_list=[0, 65535, 65536, B * H - 1], label="B*H=66000")

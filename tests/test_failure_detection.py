@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import sa3_inputs
-from sa3_testutil import bits_to_f32, qk_sf_to_canonical, rel_l2, vt_sf_to_canonical
+from sa3_testutil import assert_quantized_equal, bits_to_f32, gpu_canonical, rel_l2
 
 sa3 = pytest.importorskip("bit_quantized_attention_sa3_b200")
 
@@ -31,10 +31,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     torch.cuda.synchronize()
     assert sa3.device_status() == sa3.SA3_OK
     B, H, N, d = q.shape
-    Np = sa3.padded_len(N)
-    canon = dict(q_codes=qz.q_fp4.cpu().numpy(), k_codes=qz.k_fp4.cpu().numpy(), vt_codes=qz.vt_fp4.cpu().numpy(),
-                 q_sf=qk_sf_to_canonical(qz.q_sf.cpu().numpy(), B, H, Np, d),
-                 k_sf=qk_sf_to_canonical(qz.k_sf.cpu().numpy(), B, H, Np, d),
-                 vt_sf=vt_sf_to_canonical(qz.vt_sf.cpu().numpy(), B, H, Np, d))
-    ref = bits_to_f32(oracle.attn_fwd(canon, N, True))
+    r = oracle.quantize_qkv(q, k, v)
+    assert_quantized_equal(gpu_canonical(qz, B, H, N, N, d), r, range(B * H))
+    ref = bits_to_f32(oracle.attn_fwd(r, N, True))
     assert rel_l2(out.float().cpu().numpy(), ref) <= 2e-3

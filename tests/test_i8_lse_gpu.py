@@ -19,7 +19,8 @@ import torch
 
 import oracle
 import sa3_inputs
-from test_i8_gpu import CASES, _canon, _ids, _qkv
+from sa3_testutil import heads_of
+from test_i8_gpu import CASES, _canon, _ids, _qkv, assert_i8_equal
 
 sa3 = pytest.importorskip("bit_quantized_attention_sa3_b200")
 
@@ -49,7 +50,9 @@ def test_lse_matches_oracle(case, causal):
     torch.cuda.synchronize()
     assert sa3.device_status() == sa3.SA3_OK
     assert torch.equal(out, plain)
-    _, ref = oracle.attn_fwd_i8(_canon(qz), Nq, causal, n_kv=Nkv, return_lse=True)
+    r_q = oracle.quantize_qkv_i8(q, k, v)
+    assert_i8_equal(_canon(qz), r_q)
+    _, ref = oracle.attn_fwd_i8(r_q, Nq, causal, n_kv=Nkv, return_lse=True)
     _check_lse(lse.cpu().numpy(), ref)
     if causal and Nq > Nkv:
         assert np.isposinf(lse[:, :, : Nq - Nkv].cpu().numpy()).all()
@@ -70,16 +73,26 @@ def test_lse_full_size_sampled_units(causal):
     rng = np.random.default_rng(7)
     nqb = N // 128
     units = [(0, 0), (B * H - 1, nqb - 1)] + [(int(rng.integers(B * H)), int(rng.integers(nqb))) for _ in range(4)]
-    ref_out, ref = oracle.attn_fwd_i8(_canon(qz), N, causal, units=units, return_lse=True)
+    heads = sorted({bh for bh, _ in units})
+    pos = {bh: i for i, bh in enumerate(heads)}
+    # the oracle quantizes the sampled heads itself; they must equal the GPU's
+    r_q = oracle.quantize_qkv_i8(heads_of(q, heads), heads_of(k, heads), heads_of(v, heads))
+    g = _canon(qz)
+    for f in ("q_i8", "q_scale", "k_i8", "k_scale", "vt_f16", "k_mean"):
+        gf = g[f].reshape((B * H,) + g[f].shape[2:])[heads]
+        rf = r_q[f].reshape((len(heads),) + r_q[f].shape[2:])
+        assert np.array_equal(gf.view(np.uint8), rf.view(np.uint8)), f
+    sub = [(pos[bh], qb) for bh, qb in units]
+    ref_out, ref = oracle.attn_fwd_i8(r_q, N, causal, units=sub, return_lse=True)
     got = lse.cpu().numpy().reshape(B * H, N)
-    ref = ref.reshape(B * H, N)
+    ref = ref.reshape(len(heads), N)
     o = out.view(torch.int16).cpu().numpy().view(np.uint16).reshape(B * H, N, d)
-    ro = ref_out.reshape(B * H, N, d)
+    ro = ref_out.reshape(len(heads), N, d)
     for bh, qb in units:
         rows = slice(qb * 128, qb * 128 + 128)
-        _check_lse(got[bh, rows], ref[bh, rows])
+        _check_lse(got[bh, rows], ref[pos[bh], rows])
         a = oracle.bf16_bits_to_f32(o[bh, rows]).astype(np.float64)
-        r = oracle.bf16_bits_to_f32(ro[bh, rows]).astype(np.float64)
+        r = oracle.bf16_bits_to_f32(ro[pos[bh], rows]).astype(np.float64)
         assert np.linalg.norm(a - r) / np.linalg.norm(r) <= 2e-3
 
 

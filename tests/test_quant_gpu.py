@@ -90,13 +90,29 @@ def test_quantize_repeatable_and_ignores_workspace_contents():
 
 @pytest.mark.gpu
 def test_quantize_rejects_bad_arguments():
+    import ctypes
     q, k, v = [t.cuda() for t in sa3_inputs.make_qkv("tiny_b1h2n256d64")]
     B, H, N, d = q.shape
     out = sa3.empty_quantized(B, H, N, d)
     small = torch.empty(8, dtype=torch.uint8, device="cuda")
-    with pytest.raises(sa3.Sa3Error) as e:
+    # the binding checks the workspace first; the library checks it again
+    with pytest.raises(ValueError):
         sa3.quantize_qkv(q, k, v, out=out, workspace=small)
-    assert e.value.code == sa3.SA3_ERR_INVALID_ARG
+    st = out.struct()
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = sa3.lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(st),
+                                    small.data_ptr(), small.numel(), stream)
+    assert rc == sa3.SA3_ERR_INVALID_ARG
+    # an output or the workspace sharing bytes with an input is rejected
+    rc = sa3.lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(st),
+                                    k.data_ptr(), sa3.quant_workspace_bytes(B, H, N, d), stream)
+    assert rc == sa3.SA3_ERR_INVALID_ARG
+    alias = sa3._QKV(*[getattr(st, f) for f, _ in sa3._QKV._fields_])
+    alias.vt_fp4 = v.data_ptr() + 64
+    ws = torch.empty(sa3.quant_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+    rc = sa3.lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(alias),
+                                    ws.data_ptr(), ws.numel(), stream)
+    assert rc == sa3.SA3_ERR_INVALID_ARG
     q96 = torch.zeros((1, 1, 16, 96), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(sa3.Sa3Error) as e:
         sa3.quantize_qkv(q96, q96, q96)
