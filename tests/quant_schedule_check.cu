@@ -1,9 +1,12 @@
 // Host-side check of the quantizer's static schedule (SchedA in quant.cuh),
 // run by tests/test_quant_schedule.py: for every listed shape and grid size,
-// each Q tile, V tile and K tile is handed out exactly once, every K tile
-// belongs to the chunk it is reported in, every chunk is flushed exactly
-// once (its last tile), no job is out of range, and no CTA receives more
-// than the average plus one chunk of tiles.  Only host code runs.
+// with and without V smoothing, each Q tile and V tile is handed out
+// exactly once (V tiles: none with V smoothing, whose V tiles go to the
+// second launch), each K tile (and, with V smoothing, each V tile) exactly
+// once to a column sum, every summed tile belongs to the chunk it is
+// reported in, every chunk is flushed exactly once (its last tile), no job
+// is out of range, and no CTA receives more than the average plus one chunk
+// of tiles.  Only host code runs.
 #include "quant.cuh"
 
 #include <cstdio>
@@ -19,14 +22,16 @@ int main() {
                 const int chunk = 512 * (((N + 511) / 512 + 15) / 16);  // sa3_kmean_chunk
                 const int nchunk = (N + chunk - 1) / chunk;
                 const int tpc = chunk / 128;
+                for (int vs = 0; vs < 2; ++vs)
                 for (int G : {1, 2, 5, 37, 148, 296}) {
-                    const long long work = (long long)BH * (ntile + ntq) + (long long)BH * nchunk;
+                    const long long work = (long long)BH * (ntq + (vs ? 0 : ntile)) + (long long)BH * nchunk * (vs ? 2 : 1);
                     const int Gx = work < G ? (int)work : G;
                     std::vector<int> q(BH * ntq, 0), v(BH * ntile, 0), k(BH * ntile, 0), last(BH * nchunk, 0);
+                    std::vector<int> vsum(BH * ntile, 0), vlast(BH * nchunk, 0);
                     int maxload = 0;
                     for (int g = 0; g < Gx; ++g) {
                         sa3::quant::SchedA s;
-                        s.init(BH, ntq, ntile, nchunk, tpc, g, Gx);
+                        s.init(BH, ntq, ntile, nchunk, tpc, g, Gx, vs != 0);
                         sa3::quant::TileJob t;
                         int load = 0;
                         while (s.next(t)) {
@@ -40,12 +45,12 @@ int main() {
                             } else if (t.kind == 1) {
                                 v[t.bh * ntile + t.tile]++;
                             } else {
-                                k[t.bh * ntile + t.tile]++;
+                                (t.kind == 2 ? k : vsum)[t.bh * ntile + t.tile]++;
                                 if (t.tile / tpc != t.chunk) {
-                                    printf("K tile outside its chunk: BH=%d N=%d G=%d\n", BH, N, Gx);
+                                    printf("summed tile outside its chunk: BH=%d N=%d G=%d\n", BH, N, Gx);
                                     return 1;
                                 }
-                                if (t.last) last[t.bh * nchunk + t.chunk]++;
+                                if (t.last) (t.kind == 2 ? last : vlast)[t.bh * nchunk + t.chunk]++;
                             }
                         }
                         if (load > maxload) maxload = load;
@@ -56,16 +61,17 @@ int main() {
                             return 1;
                         }
                     for (int i = 0; i < BH * ntile; ++i)
-                        if (v[i] != 1 || k[i] != 1) {
-                            printf("V/K tile %d: %d / %d times: BH=%d N=%d G=%d\n", i, v[i], k[i], BH, N, Gx);
+                        if (v[i] != (vs ? 0 : 1) || k[i] != 1 || vsum[i] != (vs ? 1 : 0)) {
+                            printf("V/K tile %d: %d / %d / %d times: BH=%d N=%d G=%d vs=%d\n", i, v[i], k[i], vsum[i],
+                                   BH, N, Gx, vs);
                             return 1;
                         }
                     for (int i = 0; i < BH * nchunk; ++i)
-                        if (last[i] != 1) {
-                            printf("chunk %d flushed %d times: BH=%d N=%d G=%d\n", i, last[i], BH, N, Gx);
+                        if (last[i] != 1 || vlast[i] != (vs ? 1 : 0)) {
+                            printf("chunk %d flushed %d / %d times: BH=%d N=%d G=%d\n", i, last[i], vlast[i], BH, N, Gx);
                             return 1;
                         }
-                    const double avg = (double)((long long)BH * (2LL * ntile + ntq)) / Gx;
+                    const double avg = (double)((long long)BH * ((vs ? 3LL : 2LL) * ntile + ntq)) / Gx;
                     if (Gx > 2 && maxload > avg + tpc + 2) {
                         printf("imbalance: BH=%d N=%d Nq=%d G=%d max %d avg %.1f\n", BH, N, Nq, Gx, maxload, avg);
                         return 1;

@@ -1,7 +1,7 @@
 """The quantizer's static work schedule, checked on the host: the real
 SchedA of quant.cuh is compiled (nvcc, host code only; no GPU needed) into
-tests/quant_schedule_check.cu and run over 1920 shape / grid combinations,
-equal and unequal query lengths included."""
+tests/quant_schedule_check.cu and run over 3840 shape / grid / mode
+combinations, equal and unequal query lengths and V smoothing included."""
 import os
 import shutil
 import subprocess
@@ -24,4 +24,4 @@ def test_every_tile_is_scheduled_exactly_once(tmp_path):
     assert b.returncode == 0, b.stderr[-3000:]
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
-    assert r.stdout.strip() == "ok 1920 cases"
+    assert r.stdout.strip() == "ok 3840 cases"
