@@ -77,7 +77,7 @@ def _load():
         lib.oracle_quantize_qkv.restype = None
         lib.oracle_quantize_qkv.argtypes = [P, P, P, I, I, I, I, I, I, I] + [P] * 8
         lib.oracle_attn_fwd.restype = None
-        lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, I, F, I, P, P, I, P]
+        lib.oracle_attn_fwd.argtypes = [P] * 6 + [I, I, I, I, I, I, F, I, P, P, I, P, P]
         lib.oracle_attn_exact.restype = None
         lib.oracle_attn_exact.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, I, P]
         lib.oracle_f32_to_f16.restype = ctypes.c_uint16
@@ -186,13 +186,15 @@ def _units_arr(units):
 
 def attn_fwd(qz: dict, N: int, causal: bool, sm_scale: float | None = None,
              units=None, out: np.ndarray | None = None, n_kv: int | None = None,
-             p_two_level: bool = False) -> np.ndarray:
+             p_two_level: bool = False, out32: np.ndarray | None = None) -> np.ndarray:
     """Tiled FP4 attention on canonical-layout quantized operands with N
     query rows and ``n_kv`` key columns (default: qz["n_kv"] if present,
     else N).  Returns bf16 bits uint16 [B,H,N,d]; rows outside ``units``
     stay as in ``out`` (zeros by default).  ``units`` lists (b*H+h,
     q_block) pairs.  p_two_level: P pre-scaled by 2^11 before microscaling
-    (R14); qz["v_mean"], if present, is added back after O / l (R13)."""
+    (R14); qz["v_mean"], if present, is added back after O / l (R13).
+    out32 (float32 [B,H,N,d]), if given, receives the same outputs in fp32
+    just before their bf16 rounding."""
     if n_kv is None:
         n_kv = qz.get("n_kv", N)
     B, H, Np, dh = qz["q_codes"].shape
@@ -207,8 +209,10 @@ def attn_fwd(qz: dict, N: int, causal: bool, sm_scale: float | None = None,
     vm = qz.get("v_mean")
     if vm is not None:
         vm = np.ascontiguousarray(vm, dtype=np.float32)
+    if out32 is not None:
+        assert out32.dtype == np.float32 and out32.shape == out.shape and out32.flags["C_CONTIGUOUS"]
     _load().oracle_attn_fwd(*[_ptr(a) for a in arrs], B, H, N, n_kv, d, int(bool(causal)),
-                            float(sm_scale), int(bool(p_two_level)), _ptr(vm), _ptr(u), nu, _ptr(out))
+                            float(sm_scale), int(bool(p_two_level)), _ptr(vm), _ptr(u), nu, _ptr(out), _ptr(out32))
     return out
 
 

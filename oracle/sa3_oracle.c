@@ -302,13 +302,16 @@ static double deq(const uint8_t *codes, const uint8_t *sf, long elem, long sf_id
  * p_two_level: P is scaled by 2^11 before it is microscaled and the output
  * by 2^-11 after O / l (R14); v_mean (NULL: none) is added after O / l (R13).
  * units: n_units pairs (bh, q_block); NULL means every (bh, q_block).
- * out: bf16 [B*H][Nq][d]; only rows of the listed units are written. */
+ * out: bf16 [B*H][Nq][d]; only rows of the listed units are written.
+ * out32 (NULL: not wanted): the same outputs in fp32 just before the final
+ * bf16 rounding, so that a test can tell a value sitting on a bf16
+ * rounding tie from a wrong one. */
 void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
                      const uint8_t *k_codes, const uint8_t *k_sf,
                      const uint8_t *vt_codes, const uint8_t *vt_sf,
                      int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
                      int p_two_level, const float *v_mean,
-                     const int32_t *units, int n_units, uint16_t *out)
+                     const int32_t *units, int n_units, uint16_t *out, float *out32)
 {
     tables_init();
     const float p_pre = p_two_level ? 2048.0f : 1.0f;   /* 2^11, exact (R14) */
@@ -404,12 +407,14 @@ void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf,
             for (int c = 0; c < d; ++c) {
                 if (!(l > 0.0f)) {
                     out[(bh * Nq + row) * d + c] = 0;
+                    if (out32) out32[(bh * Nq + row) * d + c] = 0.0f;
                     continue;
                 }
                 float o = O[c] / l;
                 if (p_two_level) o = o * (1.0f / 2048.0f);  /* exact */
                 if (v_mean) o = o + v_mean[bh * d + c];
                 out[(bh * Nq + row) * d + c] = oracle_f32_to_bf16(o);
+                if (out32) out32[(bh * Nq + row) * d + c] = o;
             }
         }
         free(qrow);

@@ -29,7 +29,7 @@ void oracle_quantize_qkv(const uint16_t *q, const uint16_t *k, const uint16_t *v
 void oracle_attn_fwd(const uint8_t *q_codes, const uint8_t *q_sf, const uint8_t *k_codes, const uint8_t *k_sf,
                      const uint8_t *vt_codes, const uint8_t *vt_sf, int B, int H, int Nq, int Nkv, int d, int causal,
                      float sm_scale, int p_two_level, const float *v_mean, const int32_t *units, int n_units,
-                     uint16_t *out);
+                     uint16_t *out, float *out32);
 void oracle_attn_exact(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int H, int Nq, int Nkv, int d,
                        int causal, float sm_scale, const float *k_sub, const int32_t *units, int n_units,
                        double *out);
@@ -88,19 +88,20 @@ static int run_case(int B, int H, int Nq, int Nkv, int d)
     uint8_t *vc = alloc((size_t)BH * d * Np / 2), *vs = alloc((size_t)BH * d * Np / 16);
     float *km = alloc((size_t)BH * d * 4), *vm = alloc((size_t)BH * d * 4);
     uint16_t *out = alloc(nq * 2);
+    float *out32 = alloc(nq * 4);
     for (int smooth_v = 0; smooth_v < 2; ++smooth_v) {
         oracle_quantize_qkv(q, k, v, B, H, Nq, Nkv, d, 1, smooth_v, qc, qs, kc, ks, vc, vs, km, smooth_v ? vm : NULL);
         for (int causal = 0; causal < 2; ++causal)
             for (int two = 0; two < 2; ++two) {
                 memset(out, 0, nq * 2);
                 oracle_attn_fwd(qc, qs, kc, ks, vc, vs, B, H, Nq, Nkv, d, causal, sm, two, smooth_v ? vm : NULL,
-                                NULL, 0, out);
+                                NULL, 0, out, out32);
                 ok &= finite_bf16(out, nq);
             }
     }
     /* sampled units: the last Q block of the last head, then the first */
     const int32_t units[4] = {(int32_t)(BH - 1), Npq / 128 - 1, 0, 0};
-    oracle_attn_fwd(qc, qs, kc, ks, vc, vs, B, H, Nq, Nkv, d, 1, sm, 0, NULL, units, 2, out);
+    oracle_attn_fwd(qc, qs, kc, ks, vc, vs, B, H, Nq, Nkv, d, 1, sm, 0, NULL, units, 2, out, NULL);
     ok &= finite_bf16(out, nq);
 
     /* exact attention, with and without the K mean subtracted */
@@ -123,7 +124,7 @@ static int run_case(int B, int H, int Nq, int Nkv, int d)
     }
 
     free(q), free(k), free(v), free(qc), free(qs), free(kc), free(ks), free(vc), free(vs), free(km), free(vm);
-    free(out), free(ex), free(q8), free(k8), free(qsc), free(ksc), free(vt16), free(lse);
+    free(out), free(out32), free(ex), free(q8), free(k8), free(qsc), free(ksc), free(vt16), free(lse);
     if (!ok) fprintf(stderr, "non-finite output: B=%d H=%d Nq=%d Nkv=%d d=%d\n", B, H, Nq, Nkv, d);
     return ok;
 }

@@ -9,8 +9,12 @@ comparison.
 Bar: output rel-L2 <= 2e-3 against the oracle in every (head, 128-row Q
 block) compared (the GPU takes its exponentials with ex2.approx and
 accumulates in the tensor core, so P codes may flip at rounding
-boundaries; the oracle uses exp2f and fp64 sums).  The worst block and the
-worst element are printed.  The GPU is also checked against fp64 exact
+boundaries; the oracle uses exp2f and fp64 sums).  A bf16 output that is
+one ulp from the oracle's where the oracle's own fp32 value sits on the
+rounding midpoint is a rounding tie, not an error (sa3_testutil): peaked
+rows give many such values, and an ulp of the fp32 row sum, which no two
+summation orders agree on, decides them either way.  The worst block and
+the worst element are printed.  The GPU is also checked against fp64 exact
 attention of the bf16 inputs: its cosine must be within 1e-3 of the
 oracle's own cosine (the method's accuracy, not a kernel property).
 
@@ -46,13 +50,15 @@ def _chain(q, k, v, qz, out, causal, units=None, bh_list=None, sm_scale=None, la
     if units is None:
         units = [(bh, qb) for bh in heads for qb in range(nqb)]
     sub = [(pos[bh], qb) for bh, qb in units]
-    ref = bits_to_f32(oracle.attn_fwd(ref_q, Nq, causal, units=sub, sm_scale=sm_scale, p_two_level=two))[0]
+    o32 = np.zeros((1, len(heads), Nq, d), np.float32)
+    ref = bits_to_f32(oracle.attn_fwd(ref_q, Nq, causal, units=sub, sm_scale=sm_scale, p_two_level=two,
+                                      out32=o32))[0]
     ex = oracle.attn_exact(heads_of(q, heads), heads_of(k, heads), heads_of(v, heads), causal, units=sub,
                            sm_scale=sm_scale)[0]
     got = out.float().cpu().numpy().reshape(B * H, Nq, d)[heads]
     assert np.isfinite(got).all()
     live = (np.arange(Nq) + (Nkv - Nq) >= 0) if causal else None
-    worst = blockwise_rel_l2(got, ref, sub, TOL, live=live, label=label)
+    worst = blockwise_rel_l2(got, ref, sub, TOL, live=live, label=label, ref32=o32[0])
     mask = np.zeros((len(heads), Nq), bool)
     for h, qb in sub:
         mask[h, qb * 128: min(Nq, qb * 128 + 128)] = True

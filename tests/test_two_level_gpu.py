@@ -48,12 +48,13 @@ def test_two_level_matches_oracle(case, causal):
     assert np.isfinite(got).all()
     r_q = oracle.quantize_qkv(q, k, v)
     assert_quantized_equal(gpu_canonical(qz, B, H, Nq, Nkv, d), r_q, range(B * H))
-    ref = bits_to_f32(oracle.attn_fwd(r_q, Nq, causal, n_kv=Nkv, p_two_level=True))
+    o32 = np.zeros((B, H, Nq, d), np.float32)
+    ref = bits_to_f32(oracle.attn_fwd(r_q, Nq, causal, n_kv=Nkv, p_two_level=True, out32=o32))
     ex = oracle.attn_exact(q, k, v, causal)
     live = (np.arange(Nq) + (Nkv - Nq) >= 0) if causal else np.ones(Nq, bool)
     blocks = [(h, qb) for h in range(B * H) for qb in range((Nq + 127) // 128)]
     blockwise_rel_l2(got.reshape(B * H, Nq, d), ref.reshape(B * H, Nq, d), blocks, TOL, live=live,
-                     label=_ids(case))
+                     label=_ids(case), ref32=o32.reshape(B * H, Nq, d))
     g, r, e = got[:, :, live], ref[:, :, live], ex[:, :, live]
     assert cosine(g, e) >= cosine(r, e) - 1e-3
 

@@ -59,13 +59,14 @@ def test_v_smooth_matches_oracle(case, causal):
     assert np.array_equal(qz.v_mean.cpu().numpy().view(np.uint32), r_q["v_mean"].view(np.uint32))
     got = out.float().cpu().numpy()
     assert np.isfinite(got).all()
-    ref = bits_to_f32(oracle.attn_fwd(r_q, Nq, causal, n_kv=Nkv))
+    o32 = np.zeros((B, H, Nq, d), np.float32)
+    ref = bits_to_f32(oracle.attn_fwd(r_q, Nq, causal, n_kv=Nkv, out32=o32))
     live = (np.arange(Nq) + (Nkv - Nq) >= 0) if causal else np.ones(Nq, bool)
     if causal:
         assert not got[:, :, ~live].any() and not ref[:, :, ~live].any()
     blocks = [(h, qb) for h in range(B * H) for qb in range((Nq + 127) // 128)]
     blockwise_rel_l2(got.reshape(B * H, Nq, d), ref.reshape(B * H, Nq, d), blocks, TOL, live=live,
-                     label=_ids(case))
+                     label=_ids(case), ref32=o32.reshape(B * H, Nq, d))
 
 
 @pytest.mark.gpu
