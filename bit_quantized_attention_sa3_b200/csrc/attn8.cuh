@@ -30,13 +30,12 @@ namespace attn8 {
 using attn::drain_wait;
 using attn::ex2;
 using attn::kBlk;
+using attn::kSoftmaxWarps;
+using attn::kThreads;
+using attn::kWarpMma;
+using attn::kWarpProducer;
 using attn::max3f;
 using attn::warp_wait;
-
-constexpr int kSoftmaxWarps = 16;                   // 2 tiles x 2 column halves x 4 lane quadrants
-constexpr int kWarpProducer = kSoftmaxWarps;        // warp 16
-constexpr int kWarpMma = kSoftmaxWarps + 1;         // warp 17
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;  // 576 threads
 
 template <int D>
 struct Cfg {

@@ -53,9 +53,8 @@ struct AttnParams {
     float scale_log2;  // fp32(sm_scale * log2 e)
     float p_pre_log2;  // 0, or 11 for two-level P (P scaled by 2^11 before microscaling;
                        // selects the kernel instance, whose exponent is fixed)
-    int npairs;        // 8-bit kernel: Q-tile pairs per head (set by the launcher)
-    int pair_units;    // 8-bit kernel: work units that are pairs; the rest are single tiles
-    int hg;            // FP4 kernel: heads per group of its persistent work list (set by the launcher)
+    int npairs;        // Q-tile pairs per head (set by the launcher)
+    int pair_units;    // work units that are pairs; the rest are single tiles
 };
 
 // Host: raise Kernel's dynamic shared memory limit once per device (the
