@@ -70,11 +70,13 @@ def parse():
                          "(sa3_*_lens; causal aligns the last query with the last key)")
     ap.add_argument("--p-two-level", action="store_true",
                     help="fp4 only: P pre-scaled by 2^11 before it is microscaled (SA3_P_TWO_LEVEL)")
+    ap.add_argument("--v-smooth", action="store_true",
+                    help="fp4 only: V smoothed like K, its mean added back after O / l (SA3_V_SMOOTH)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
     args = ap.parse_args()
-    if args.p_two_level and args.variant != "fp4":
-        ap.error("--p-two-level applies to the fp4 variant only")
+    if (args.p_two_level or args.v_smooth) and args.variant != "fp4":
+        ap.error("--p-two-level and --v-smooth apply to the fp4 variant only")
     if args.nq < 0:
         ap.error("--nq must be positive")
     return args
@@ -213,7 +215,7 @@ def fp4_peak_probe(sa3, dev, iters=16384):
     return res
 
 
-def accuracy_sample(w, q, k, v, out, causal, two=False, nunits=6):
+def accuracy_sample(w, q, k, v, out, causal, two=False, vsm=False, nunits=6):
     """The output's accuracy on a seeded sample of (head, Q block) units: the
     oracle quantizes those heads itself and attends on its own operands
     (worst per-block rel-L2 of the GPU output against it), and the fp64
@@ -233,7 +235,7 @@ def accuracy_sample(w, q, k, v, out, causal, two=False, nunits=6):
         B, H, n, d = t.shape
         return t.reshape(B * H, n, d)[heads].reshape(1, len(heads), n, d).contiguous()
     qs, ks, vs = hd(q), hd(k), hd(v)
-    rq = oracle.quantize_qkv(qs, ks, vs)
+    rq = oracle.quantize_qkv(qs, ks, vs, smooth_v=vsm)
     ref = oracle.bf16_bits_to_f32(oracle.attn_fwd(rq, Nq, causal, units=sub, p_two_level=two))[0]
     ex = oracle.attn_exact(qs, ks, vs, causal, units=sub)[0]
     got = out.float().cpu().numpy().reshape(w.B * w.H, Nq, w.d)[heads]
@@ -288,12 +290,19 @@ def run_sa3(args, rank, world, local):
     B, H, N, d, causal = w.B, w.H, w.N, w.d, w.causal
     Nq = args.nq or N
     two = bool(args.p_two_level)
+    vsm = bool(args.v_smooth)
     q_h, k_h, v_h = make_inputs(w, Nq, seed=rank)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     i8 = args.variant in ("i8", "i8_train")
     train = args.variant == "i8_train"
-    empty_q = sa3.empty_quantized_i8 if i8 else sa3.empty_quantized
-    quantize = sa3.quantize_qkv_i8 if i8 else sa3.quantize_qkv
+    if i8:
+        empty_q, quantize = sa3.empty_quantized_i8, sa3.quantize_qkv_i8
+    else:
+        def empty_q(B, H, N, d, dev, Nq):
+            return sa3.empty_quantized(B, H, N, d, dev, Nq=Nq, v_smooth=vsm)
+
+        def quantize(q, k, v, out, workspace, stream=None):
+            return sa3.quantize_qkv(q, k, v, out=out, workspace=workspace, stream=stream, v_smooth=vsm)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev) if train else None
 
     def attend(qz, causal, out, stream=None, lse=lse):
@@ -301,7 +310,7 @@ def run_sa3(args, rank, world, local):
             return sa3.attn_fwd_i8(qz, causal=causal, out=out, stream=stream, lse=lse)
         return sa3.attn_fwd(qz, causal=causal, out=out, stream=stream, p_two_level=two)
     qz = empty_q(B, H, N, d, dev, Nq=Nq)
-    ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d, vsm)), dtype=torch.uint8, device=dev)
     out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -479,14 +488,16 @@ def run_sa3(args, rank, world, local):
         line["config"]["ops"] = "4*d per (query, key) pair the mask leaves"
     if two:
         line["config"]["p_two_level"] = True
+    if vsm:
+        line["config"]["v_smooth"] = True
     if world == 1 and not args.skip_cpu_baseline:
         if not i8:
-            line["accuracy"] = accuracy_sample(w, q_h, k_h, v_h, out, causal, two=two)
-        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8, train=train, two=two)
+            line["accuracy"] = accuracy_sample(w, q_h, k_h, v_h, out, causal, two=two, vsm=vsm)
+        line["cpu_baseline"] = cpu_baseline(w, q_h, k_h, v_h, budget_s=15.0, i8=i8, train=train, two=two, vsm=vsm)
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=False, two=False):
+def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=False, two=False, vsm=False):
     """The oracle, as it stands, on the host cores: full quantization plus
     attention for a seeded sample of Q blocks; the full-job time is
     extrapolated from the sampled blocks, each weighted by the KV blocks it
@@ -496,7 +507,7 @@ def cpu_baseline(w, q, k, v, budget_s=15.0, units_cap=None, i8=False, train=Fals
     oracle.build()
     Nq, N = q.shape[2], k.shape[2]
     t0 = time.perf_counter()
-    qz = (oracle.quantize_qkv_i8 if i8 else oracle.quantize_qkv)(q, k, v)
+    qz = oracle.quantize_qkv_i8(q, k, v) if i8 else oracle.quantize_qkv(q, k, v, smooth_v=vsm)
     t_quant = time.perf_counter() - t0
     nqb, nkv = (Nq + 127) // 128, (N + 127) // 128
     total_units = w.B * w.H * nqb
@@ -544,7 +555,8 @@ def run_reference(args, rank, world):
     i8, train = args.variant in ("i8", "i8_train"), args.variant == "i8_train"
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        cb = cpu_baseline(w, q, k, v, budget_s=budget, i8=i8, train=train, two=bool(args.p_two_level))
+        cb = cpu_baseline(w, q, k, v, budget_s=budget, i8=i8, train=train, two=bool(args.p_two_level),
+                          vsm=bool(args.v_smooth))
         if i >= args.warmup:
             per_step.append(cb)
             wall.append(time.perf_counter() - t0)
@@ -563,6 +575,7 @@ def run_reference(args, rank, world):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "variant": args.variant, **({"Nq": Nq} if Nq != w.N else {}),
                    **({"p_two_level": True} if args.p_two_level else {}),
+                   **({"v_smooth": True} if args.v_smooth else {}),
                    "step": "oracle quantize + tiled attention (sampled, extrapolated)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"]},

@@ -160,10 +160,16 @@ int sa3_quantize_qkv(const void *q, const void *k, const void *v,
  *
  * Accuracy: the recipe above is followed step by step, but not to the bit.
  * The exponentials use the hardware's approximate exp2.  1/s is folded into
- * the exponent: y = 2^(t - m' + log2(1/s)), rounded at the size of m'.
- * Tensor-core sums run in their own order.  So a P code may differ from
- * the recipe's where the value sits at a rounding boundary.  Outputs stay
- * within relative L2 2e-3 of the step-by-step recipe.
+ * the exponent: y = 2^(S*c + (log2(1/s) - m')) from one fused multiply-add,
+ * and l is formed as sum_b s_b * sum(y).  Tensor-core sums run in their own
+ * order.  So a P code may differ from the recipe's where the value sits at
+ * a rounding boundary, and an output may land one bf16 ulp away where the
+ * recipe's own fp32 value sits on a rounding midpoint (peaked rows, whose
+ * values are short binary fractions, have many).  Rounding ties aside, the
+ * outputs were measured within relative L2 1.4e-3 of the recipe in every
+ * 128-row block, for softmax scales up to 1024/sqrt(d) (logits up to about
+ * 10^6) on LLM- and video-DiT-shaped inputs, both masks; the parity tests
+ * hold every block to 2e-3.  Scaled logits must be finite in fp32.
  *
  * in       : quantized operands from sa3_quantize_qkv for the same shape.
  * causal   : 0 or 1 (mask col > row, rows and columns both from 0).
