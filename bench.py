@@ -72,11 +72,14 @@ def parse():
                     help="fp4 only: P pre-scaled by 2^11 before it is microscaled (SA3_P_TWO_LEVEL)")
     ap.add_argument("--v-smooth", action="store_true",
                     help="fp4 only: V smoothed like K, its mean added back after O / l (SA3_V_SMOOTH)")
+    ap.add_argument("--q-on-load", action="store_true",
+                    help="fp4 only: the quantizer skips Q and the attention kernel quantizes the bf16 Q "
+                         "itself (SA3_SKIP_Q + SA3_Q_ON_LOAD); same output bits")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (for profiler runs)")
     args = ap.parse_args()
-    if (args.p_two_level or args.v_smooth) and args.variant != "fp4":
-        ap.error("--p-two-level and --v-smooth apply to the fp4 variant only")
+    if (args.p_two_level or args.v_smooth or args.q_on_load) and args.variant != "fp4":
+        ap.error("--p-two-level, --v-smooth and --q-on-load apply to the fp4 variant only")
     if args.nq < 0:
         ap.error("--nq must be positive")
     return args
@@ -291,6 +294,7 @@ def run_sa3(args, rank, world, local):
     Nq = args.nq or N
     two = bool(args.p_two_level)
     vsm = bool(args.v_smooth)
+    qload = bool(args.q_on_load)
     q_h, k_h, v_h = make_inputs(w, Nq, seed=rank)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     i8 = args.variant in ("i8", "i8_train")
@@ -299,16 +303,18 @@ def run_sa3(args, rank, world, local):
         empty_q, quantize = sa3.empty_quantized_i8, sa3.quantize_qkv_i8
     else:
         def empty_q(B, H, N, d, dev, Nq):
-            return sa3.empty_quantized(B, H, N, d, dev, Nq=Nq, v_smooth=vsm)
+            return sa3.empty_quantized(B, H, N, d, dev, Nq=Nq, v_smooth=vsm, skip_q=qload)
 
         def quantize(q, k, v, out, workspace, stream=None):
-            return sa3.quantize_qkv(q, k, v, out=out, workspace=workspace, stream=stream, v_smooth=vsm)
+            return sa3.quantize_qkv(q, k, v, out=out, workspace=workspace, stream=stream, v_smooth=vsm,
+                                    skip_q=qload)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev) if train else None
 
-    def attend(qz, causal, out, stream=None, lse=lse):
+    def attend(qz, causal, out, stream=None, lse=lse, qsrc=None):
         if i8:
             return sa3.attn_fwd_i8(qz, causal=causal, out=out, stream=stream, lse=lse)
-        return sa3.attn_fwd(qz, causal=causal, out=out, stream=stream, p_two_level=two)
+        return sa3.attn_fwd(qz, causal=causal, out=out, stream=stream, p_two_level=two,
+                            q=qsrc if qload else None)
     qz = empty_q(B, H, N, d, dev, Nq=Nq)
     ws = torch.empty(max(16, sa3.quant_workspace_bytes(B, H, N, d, vsm)), dtype=torch.uint8, device=dev)
     out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=dev)
@@ -323,7 +329,7 @@ def run_sa3(args, rank, world, local):
 
     def step():
         quantize(q, k, v, out=qz, workspace=ws)
-        attend(qz, causal=causal, out=out)
+        attend(qz, causal=causal, out=out, qsrc=q)
 
     for _ in range(args.warmup):
         step()
@@ -342,7 +348,7 @@ def run_sa3(args, rank, world, local):
             ev[i][0].record(stream)
             quantize(q, k, v, out=qz, workspace=ws)
             ev[i][1].record(stream)
-            attend(qz, causal=causal, out=out)
+            attend(qz, causal=causal, out=out, qsrc=q)
             ev[i][2].record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -382,7 +388,7 @@ def run_sa3(args, rank, world, local):
                 b["ready"].record(up_s)
             stream.wait_event(b["ready"])
             quantize(b["q"], b["k"], b["v"], out=b["qz"], workspace=b["ws"], stream=stream)
-            attend(b["qz"], causal=causal, out=b["out"], stream=stream, lse=b["lse"])
+            attend(b["qz"], causal=causal, out=b["out"], stream=stream, lse=b["lse"], qsrc=b["q"])
             b["done"].record(stream)
             down_s.wait_event(b["done"])
             with torch.cuda.stream(down_s):
@@ -427,7 +433,8 @@ def run_sa3(args, rank, world, local):
     ops = attn_ops(w, Nq)
     achieved = ops / (t_attn * 1e-3) / 1e12
     Np, Npq = sa3.padded_len(N), sa3.padded_len(Nq)
-    rd = B * H * d * 2 * (Nq + 2 * N)           # bf16 q, k, v read once
+    nq_quant = 0 if qload else Nq               # Q on load: the quantizer reads and writes no Q
+    rd = B * H * d * 2 * (nq_quant + 2 * N)     # bf16 q, k, v read once
     if i8:
         # half the ops at the int8 rate (2x bf16, nominal), half at the fp16 rate
         peak = pk["bf16_tflops"] * 4.0 / 3.0
@@ -440,7 +447,8 @@ def run_sa3(args, rank, world, local):
         peak_src = (f"measured in this run: {probe['how']} (N=128 {probe['n128_tops']}, "
                     f"N=256 {probe['n256_tops']} TOPS)")
         peak_rule = pk["bf16_tflops"] * FP4_PER_BF16
-        qk_bytes = rd + B * H * d * (Npq + 2 * Np) // 2 + B * H * d * (Npq + 2 * Np) // 16
+        npq_quant = 0 if qload else Npq
+        qk_bytes = rd + B * H * d * (npq_quant + 2 * Np) // 2 + B * H * d * (npq_quant + 2 * Np) // 16
         dtype = "fp4-e2m1 (ue4m3 scales, fp32 accumulate)"
         kernel = "attn_fwd_kernel<%d>" % d
         traffic = profiled_traffic("bit_quantized_attention_sa3_b200/csrc/attn.cuh",
@@ -490,6 +498,9 @@ def run_sa3(args, rank, world, local):
         line["config"]["p_two_level"] = True
     if vsm:
         line["config"]["v_smooth"] = True
+    if qload:
+        line["config"]["q_on_load"] = True
+        line["config"]["step"] = "sa3_quantize_qkv_ex (SA3_SKIP_Q) + sa3_attn_fwd_ex (SA3_Q_ON_LOAD)"
     if world == 1 and not args.skip_cpu_baseline:
         if not i8:
             line["accuracy"] = accuracy_sample(w, q_h, k_h, v_h, out, causal, two=two, vsm=vsm)

@@ -38,6 +38,8 @@ SA3_ERR_CUDA = 3
 SA3_ERR_TIMEOUT = 4
 SA3_P_TWO_LEVEL = 1
 SA3_V_SMOOTH = 2
+SA3_SKIP_Q = 4
+SA3_Q_ON_LOAD = 8
 _NAMES = {0: "SA3_OK", 1: "SA3_ERR_INVALID_ARG", 2: "SA3_ERR_UNSUPPORTED", 3: "SA3_ERR_CUDA",
           4: "SA3_ERR_TIMEOUT"}
 
@@ -100,7 +102,7 @@ def lib() -> ctypes.CDLL:
             L.sa3_quantize_qkv_ex.argtypes = [P, P, P, I, I, I, I, I, ctypes.c_uint, ctypes.POINTER(_QKV), P, P,
                                               ctypes.c_size_t, P]
             L.sa3_attn_fwd_ex.restype = I
-            L.sa3_attn_fwd_ex.argtypes = [ctypes.POINTER(_QKV), P, I, I, I, I, I, I, F, ctypes.c_uint, P, P]
+            L.sa3_attn_fwd_ex.argtypes = [ctypes.POINTER(_QKV), P, P, I, I, I, I, I, I, F, ctypes.c_uint, P, P]
             L.sa3_probe_fp4_mma.restype = I
             L.sa3_probe_fp4_mma.argtypes = [I, I, I, P, P]
             _lib = L
@@ -130,9 +132,11 @@ def quant_workspace_bytes(B: int, H: int, N: int, d: int, v_smooth: bool = False
 @dataclasses.dataclass
 class QuantizedQKV:
     """Device buffers of the quantized operands (layouts: include/sa3.h).
-    N is the key/value length; Nq the query length (None: equal to N)."""
-    q_fp4: torch.Tensor   # u8 [B,H,Np(Nq),d/2]
-    q_sf: torch.Tensor    # u8, 128x4 scale atoms
+    N is the key/value length; Nq the query length (None: equal to N).
+    q_fp4 and q_sf are None when Q was left to the attention kernel
+    (skip_q: it quantizes Q on load)."""
+    q_fp4: torch.Tensor | None   # u8 [B,H,Np(Nq),d/2]
+    q_sf: torch.Tensor | None    # u8, 128x4 scale atoms
     k_fp4: torch.Tensor   # u8 [B,H,Np,d/2]
     k_sf: torch.Tensor
     vt_fp4: torch.Tensor  # u8 [B,H,d,Np/2]
@@ -151,7 +155,7 @@ class QuantizedQKV:
 
     @property
     def device(self) -> torch.device:
-        return self.q_fp4.device
+        return self.k_fp4.device
 
     def check(self, device: torch.device | None = None) -> None:
         """Raise ValueError unless every buffer is a contiguous tensor of the
@@ -160,8 +164,11 @@ class QuantizedQKV:
         dev = self.device if device is None else device
         Npq, Np = padded_len(self.n_q), padded_len(self.N)
         B, H, d = self.B, self.H, self.d
-        _check_buffer(self.q_fp4, "q_fp4", torch.uint8, B * H * Npq * d // 2, dev)
-        _check_buffer(self.q_sf, "q_sf", torch.uint8, B * H * Npq * d // 16, dev)
+        if (self.q_fp4 is None) != (self.q_sf is None):
+            raise ValueError("q_fp4 and q_sf must both be given or both be None")
+        if self.q_fp4 is not None:
+            _check_buffer(self.q_fp4, "q_fp4", torch.uint8, B * H * Npq * d // 2, dev)
+            _check_buffer(self.q_sf, "q_sf", torch.uint8, B * H * Npq * d // 16, dev)
         _check_buffer(self.k_fp4, "k_fp4", torch.uint8, B * H * Np * d // 2, dev)
         _check_buffer(self.k_sf, "k_sf", torch.uint8, B * H * Np * d // 16, dev)
         _check_buffer(self.vt_fp4, "vt_fp4", torch.uint8, B * H * d * Np // 2, dev)
@@ -171,20 +178,24 @@ class QuantizedQKV:
             _check_buffer(self.v_mean, "v_mean", torch.float32, B * H * d, dev)
 
     def struct(self) -> _QKV:
-        return _QKV(self.q_fp4.data_ptr(), self.q_sf.data_ptr(), self.k_fp4.data_ptr(),
+        qp = 0 if self.q_fp4 is None else self.q_fp4.data_ptr()
+        qs = 0 if self.q_sf is None else self.q_sf.data_ptr()
+        return _QKV(qp, qs, self.k_fp4.data_ptr(),
                     self.k_sf.data_ptr(), self.vt_fp4.data_ptr(), self.vt_sf.data_ptr(),
                     self.k_mean.data_ptr())
 
 
 def empty_quantized(B: int, H: int, N: int, d: int, device="cuda", Nq: int | None = None,
-                    v_smooth: bool = False) -> QuantizedQKV:
+                    v_smooth: bool = False, skip_q: bool = False) -> QuantizedQKV:
     """Buffers for keys/values of length N and queries of length Nq (default N);
-    with v_smooth also the mean of V (V smoothing)."""
+    with v_smooth also the mean of V (V smoothing); with skip_q no Q buffers
+    (Q quantized on load by the attention kernel)."""
     Np = padded_len(N)
     Npq = padded_len(N if Nq is None else Nq)
     u8 = dict(dtype=torch.uint8, device=device)
     return QuantizedQKV(
-        q_fp4=torch.empty((B, H, Npq, d // 2), **u8), q_sf=torch.empty(B * H * Npq * d // 16, **u8),
+        q_fp4=None if skip_q else torch.empty((B, H, Npq, d // 2), **u8),
+        q_sf=None if skip_q else torch.empty(B * H * Npq * d // 16, **u8),
         k_fp4=torch.empty((B, H, Np, d // 2), **u8), k_sf=torch.empty(B * H * Np * d // 16, **u8),
         vt_fp4=torch.empty((B, H, d, Np // 2), **u8), vt_sf=torch.empty(B * H * Np * 8, **u8),
         k_mean=torch.empty((B, H, d), dtype=torch.float32, device=device), B=B, H=H, N=N, d=d,
@@ -251,22 +262,25 @@ def _check_out(out: torch.Tensor, shape: tuple, device: torch.device) -> None:
 
 def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  out: QuantizedQKV | None = None, workspace: torch.Tensor | None = None,
-                 stream=None, v_smooth: bool = False) -> QuantizedQKV:
+                 stream=None, v_smooth: bool = False, skip_q: bool = False) -> QuantizedQKV:
     """sa3_quantize_qkv: K smoothing, then E2M1 codes + E4M3 scales of Q, K, V.
     q is [B,H,Nq,d]; k and v are [B,H,N,d] (N may differ from Nq:
     sa3_quantize_qkv_lens).  v_smooth: V is smoothed like K and its mean
     kept in the result (sa3_quantize_qkv_ex with SA3_V_SMOOTH); attn_fwd
-    then adds it back."""
+    then adds it back.  skip_q: Q is not quantized here (SA3_SKIP_Q); pass
+    q to attn_fwd, which quantizes it on load."""
     dev = _check_qkv(q, k, v)
     B, H, Nq, d = q.shape
     N = k.shape[2]
     with torch.cuda.device(dev):
         if out is None:
-            out = empty_quantized(B, H, N, d, dev, Nq=Nq, v_smooth=v_smooth)
+            out = empty_quantized(B, H, N, d, dev, Nq=Nq, v_smooth=v_smooth, skip_q=skip_q)
         if (out.B, out.H, out.d, out.n_q, out.N) != (B, H, d, Nq, N):
             raise ValueError("out was sized for another shape")
         if v_smooth != (out.v_mean is not None):
             raise ValueError("out must hold v_mean exactly when v_smooth is set")
+        if not skip_q and out.q_fp4 is None:
+            raise ValueError("out has no Q buffers: quantize with skip_q=True")
         out.check(dev)
         nbytes = quant_workspace_bytes(B, H, N, d, v_smooth)
         if workspace is None:
@@ -274,10 +288,11 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         ws_bytes = _check_workspace(workspace, nbytes, dev)
         sp = _stream_ptr(stream, dev)
         st = out.struct()
-        if v_smooth:
-            rc = lib().sa3_quantize_qkv_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, Nq, N, d, SA3_V_SMOOTH,
-                                           ctypes.byref(st), out.v_mean.data_ptr(), workspace.data_ptr(), ws_bytes,
-                                           sp)
+        if v_smooth or skip_q:
+            flags = (SA3_V_SMOOTH if v_smooth else 0) | (SA3_SKIP_Q if skip_q else 0)
+            rc = lib().sa3_quantize_qkv_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, Nq, N, d, flags,
+                                           ctypes.byref(st), out.v_mean.data_ptr() if v_smooth else None,
+                                           workspace.data_ptr(), ws_bytes, sp)
         elif Nq == N:
             rc = lib().sa3_quantize_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, ctypes.byref(st),
                                         workspace.data_ptr(), ws_bytes, sp)
@@ -290,18 +305,27 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 
 def attn_fwd(qz: QuantizedQKV, causal: bool = False, sm_scale: float | None = None,
-             out: torch.Tensor | None = None, stream=None, p_two_level: bool = False) -> torch.Tensor:
+             out: torch.Tensor | None = None, stream=None, p_two_level: bool = False,
+             q: torch.Tensor | None = None) -> torch.Tensor:
     """sa3_attn_fwd: FP4 attention of quantized operands; bf16 [B,H,Nq,d].
     With Nq != N (sa3_attn_fwd_lens) the causal mask aligns the last query
     with the last key; a row that sees no key is 0.  p_two_level: P scaled
     by 2^11 before it is microscaled (SA3_P_TWO_LEVEL).  Operands quantized
     with v_smooth carry V's mean, which is added back (sa3_attn_fwd_ex with
-    SA3_V_SMOOTH)."""
+    SA3_V_SMOOTH).  q (bf16 [B,H,Nq,d]): the kernel quantizes Q on load
+    (SA3_Q_ON_LOAD) instead of reading qz's Q codes; required when qz was
+    made with skip_q."""
     B, H, N, d, Nq = qz.B, qz.H, qz.N, qz.d, qz.n_q
     dev = qz.device
     if dev.type != "cuda":
         raise ValueError("the quantized operands must be CUDA tensors")
     qz.check(dev)
+    if q is not None:
+        _check_input(q, "q")
+        if tuple(q.shape) != (B, H, Nq, d) or q.device != dev:
+            raise ValueError("q must be bf16 [B,H,Nq,d] on the operands' device")
+    elif qz.q_fp4 is None:
+        raise ValueError("qz holds no Q codes (skip_q): pass q to quantize it on load")
     with torch.cuda.device(dev):
         if out is None:
             out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=dev)
@@ -310,10 +334,12 @@ def attn_fwd(qz: QuantizedQKV, causal: bool = False, sm_scale: float | None = No
         scale = 0.0 if sm_scale is None else float(sm_scale)
         sp = _stream_ptr(stream, dev)
         st = qz.struct()
-        if qz.v_mean is not None:
-            flags = SA3_V_SMOOTH | (SA3_P_TWO_LEVEL if p_two_level else 0)
-            rc = lib().sa3_attn_fwd_ex(ctypes.byref(st), qz.v_mean.data_ptr(), B, H, Nq, N, d, int(bool(causal)),
-                                       scale, flags, out.data_ptr(), sp)
+        if qz.v_mean is not None or q is not None:
+            flags = ((SA3_V_SMOOTH if qz.v_mean is not None else 0) | (SA3_P_TWO_LEVEL if p_two_level else 0)
+                     | (SA3_Q_ON_LOAD if q is not None else 0))
+            rc = lib().sa3_attn_fwd_ex(ctypes.byref(st), q.data_ptr() if q is not None else None,
+                                       qz.v_mean.data_ptr() if qz.v_mean is not None else None, B, H, Nq, N, d,
+                                       int(bool(causal)), scale, flags, out.data_ptr(), sp)
         elif Nq == N and not p_two_level:
             rc = lib().sa3_attn_fwd(ctypes.byref(st), B, H, N, d, int(bool(causal)), scale, out.data_ptr(), sp)
         else:

@@ -32,6 +32,7 @@
 // pipes (the bottleneck on B200) stay busy.
 #pragma once
 
+#include "quant.cuh"
 #include "sa3_internal.h"
 #include "sm100.cuh"
 
@@ -45,7 +46,7 @@ constexpr int kWarpProducer = kSoftmaxWarps;     // warp 16
 constexpr int kWarpMma = kSoftmaxWarps + 1;      // warp 17
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;  // 576 threads (at most 112 registers each)
 
-constexpr int kBarCountBytes = (17 + 2 * kStages) * 8;  // barrier slots below
+constexpr int kBarCountBytes = (18 + 2 * kStages) * 8;  // barrier slots below
 
 template <int D>
 struct Cfg {
@@ -79,6 +80,14 @@ struct Cfg {
     static constexpr int oXl = oXch + 4096;            // row sums [2 tiles][2 halves][128]
     static constexpr int oBar = oXl + 2048;
     static constexpr int kSmemBytes = oBar + 256 + 1024;
+    // Q quantized on load (kQLoad instances only): bf16 staging of the two Q
+    // tiles (D/64 boxes of 64 channels x 128 tokens each, 128-byte swizzle,
+    // as the quantizer stages them) and 1/s per E4M3 scale code
+    static constexpr int kQbfBytes = kBlk * D * 2;
+    static constexpr int oQbf = al(oBar + 256);
+    static constexpr int oRcp = oQbf + 2 * kQbfBytes;
+    static constexpr int kSmemBytesQL = oRcp + 1024 + 1024;
+    static_assert(kSmemBytesQL <= 227 * 1024, "shared memory budget (Q on load)");
     // TMEM columns
     static constexpr uint32_t tS = 0;
     static constexpr uint32_t tO0 = 128;
@@ -104,7 +113,8 @@ enum : int {
     kBarPvDone = 6 + 2 * kStages,    // 2
     kBarDrain = 8 + 2 * kStages,     // 1
     kBarXch = 9 + 2 * kStages,       // 8: [tile][lane quadrant], 64 arrivals
-    kBarCount = 17 + 2 * kStages
+    kBarQReady = 17 + 2 * kStages,   // 1 (Q on load): the 512 softmax threads have quantized Q
+    kBarCount = 18 + 2 * kStages
 };
 static_assert(kBarCount * 8 == kBarCountBytes, "barrier slots");
 
@@ -147,11 +157,40 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// Quantizes one staged bf16 Q tile in shared memory (this thread: token row
+// t/2, channel half t%2 of the tile's 256 threads) into the layout the MMA
+// reads: E2M1 codes in 64-byte (D = 128) or 32-byte (D = 64) swizzled
+// K-major rows, scales in 512-byte atoms.  The blocks are quantized by the
+// quantizer's own routine; rows past Nq arrive as zeros and get code 0,
+// scale 0.
+template <int D>
+__device__ __forceinline__ void quantize_q_tile(const uint8_t *__restrict__ stage, const float *__restrict__ rcp_lut,
+                                                uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, int t) {
+    const int row = t >> 1;
+    const int part = t & 1;
+    uint32_t cw[D / 16];
+    const uint32_t scw = quant::row_part_codes<D>(stage, row, part, false, nullptr, rcp_lut, cw);
+    if constexpr (D == 128) {
+        // 64-byte rows; 16-byte chunks 2*part, 2*part+1, chunk index XOR (row/2)%4
+        uint8_t *prow = codes + row * 64;
+        const int sw = (row >> 1) & 3;
+        *reinterpret_cast<uint4 *>(prow + (((2 * part) ^ sw) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4 *>(prow + (((2 * part + 1) ^ sw) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        *reinterpret_cast<uint32_t *>(sf + part * 512 + quant::atom_off(row, 0)) = scw;
+    } else {
+        // 32-byte rows; 16-byte chunk `part`, chunk index XOR (row/4)%2
+        *reinterpret_cast<uint4 *>(codes + row * 32 + ((part ^ ((row >> 2) & 1)) << 4)) =
+            make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint16_t *>(sf + quant::atom_off(row, 2 * part)) = static_cast<uint16_t>(scw);
+    }
+}
+
 // kCross: query and key/value lengths differ (bottom-right causal offset,
 // rows that may see no key).  kTwo: P is pre-scaled by 2^11 before it is
-// microscaled (two-level P).  Each term is compiled only into the instances
-// that use it.
-template <int D, bool kCross, bool kTwo>
+// microscaled (two-level P).  kQLoad: Q arrives as bf16 and the softmax
+// warps quantize it before the first S (tm_q is then the 3-D bf16 map).
+// Each term is compiled only into the instances that use it.
+template <int D, bool kCross, bool kTwo, bool kQLoad>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -209,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bars + kBarPvDone + 1, 1);
         mbar_init(bars + kBarDrain, 1);
         for (int x = 0; x < 8; ++x) mbar_init(bars + kBarXch + x, 64);
+        mbar_init(bars + kBarQReady, 16 * 32);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -225,6 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float pre = kTwo ? 11.0f : 0.0f;
         reinterpret_cast<float *>(base + C::oLut)[threadIdx.x] = unit ? pre : pre - log2f(v);
         reinterpret_cast<float *>(base + C::oLut)[256 + threadIdx.x] = unit ? 1.0f : v;
+        if constexpr (kQLoad)
+            reinterpret_cast<float *>(base + C::oRcp)[threadIdx.x] = unit ? 0.0f : __frcp_rn(v);  // 1/s, exact
     }
     if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -233,6 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Launched as a programmatic dependent: everything above overlaps the
+    // tail of the kernel before (the quantizer); every global read below
+    // comes after it has completed
+    pdl_wait();
     const uint32_t tmem = *tmem_slot;
     const float *lg_lut = reinterpret_cast<const float *>(base + C::oLut);
     const float *sv_lut = lg_lut + 256;
@@ -245,13 +291,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tm_k);
             prefetch_tensormap(&tm_v);
             uint64_t *bq = bars + kBarQ;
-            mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * (C::kQBytes + C::kSfBytes));
-            tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Npq + tile0 * kBlk, bq);
-            bulk_load(base + C::oQsf0, p.q_sf + static_cast<size_t>(bh * nqt + tile0) * C::kSfBytes, C::kSfBytes, bq);
-            if (valid1) {
-                tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Npq + tile1 * kBlk, bq);
-                bulk_load(base + C::oQsf1, p.q_sf + static_cast<size_t>(bh * nqt + tile1) * C::kSfBytes, C::kSfBytes,
+            if constexpr (kQLoad) {
+                // bf16 Q tiles, boxes of 64 channels x 128 tokens (tokens past Nq read as 0)
+                const uint64_t pol = l2_policy_evict_first();
+                mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * C::kQbfBytes);
+                for (int i = 0; i <= static_cast<int>(valid1); ++i)
+#pragma unroll
+                    for (int b = 0; b < D / 64; ++b)
+                        tma_load_3d_hint(base + C::oQbf + i * C::kQbfBytes + b * (kBlk * 128), &tm_q, b * 64,
+                                         (i ? tile1 : tile0) * kBlk, bh, bq, pol);
+            } else {
+                mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * (C::kQBytes + C::kSfBytes));
+                tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Npq + tile0 * kBlk, bq);
+                bulk_load(base + C::oQsf0, p.q_sf + static_cast<size_t>(bh * nqt + tile0) * C::kSfBytes, C::kSfBytes,
                           bq);
+                if (valid1) {
+                    tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Npq + tile1 * kBlk, bq);
+                    bulk_load(base + C::oQsf1, p.q_sf + static_cast<size_t>(bh * nqt + tile1) * C::kSfBytes,
+                              C::kSfBytes, bq);
+                }
             }
             int issued = 0;
             for (int j = 0; j < nmax; ++j) {
@@ -344,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
 
-            bool ok = mbar_wait(bars + kBarQ, 0, abort_flag);
+            bool ok = mbar_wait(bars + (kQLoad ? kBarQReady : kBarQ), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
@@ -415,7 +473,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = -INFINITY;
         float l = 0.0f;
         bool ok = true;
-        for (int j = 0; j < n_i; ++j) {
+        if constexpr (kQLoad) {
+            // Q on load: the 256 threads of tile i quantize its staged bf16
+            // tile into the Q code and scale buffers the MMA reads
+            ok = warp_wait(bars + kBarQ, 0, abort_flag);
+            if (ok && (i == 0 || valid1))
+                quantize_q_tile<D>(base + C::oQbf + i * C::kQbfBytes, reinterpret_cast<const float *>(base + C::oRcp),
+                                   base + (i ? C::oQ1 : C::oQ0), base + (i ? C::oQsf1 : C::oQsf0),
+                                   static_cast<int>(threadIdx.x) & 255);
+            fence_proxy_async_smem();
+            mbar_arrive(bars + kBarQReady);
+        }
+        for (int j = 0; ok && j < n_i; ++j) {
             if (!warp_wait(bars + kBarSFull + i, j & 1, abort_flag)) {
                 ok = false;
                 break;
@@ -630,18 +699,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
-cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                     cudaStream_t stream) {
+template <int D, bool kQLoad>
+cudaError_t launch_dq(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                      cudaStream_t stream) {
     using C = Cfg<D>;
+    constexpr int smem = kQLoad ? C::kSmemBytesQL : C::kSmemBytes;
     const bool cross = p.Nq != p.N;
     const bool two = p.p_pre_log2 != 0.0f;
-    auto kernel = cross ? (two ? attn_fwd_kernel<D, true, true> : attn_fwd_kernel<D, true, false>)
-                        : (two ? attn_fwd_kernel<D, false, true> : attn_fwd_kernel<D, false, false>);
-    cudaError_t e = cross ? (two ? smem_attr_once<attn_fwd_kernel<D, true, true>>(C::kSmemBytes)
-                                 : smem_attr_once<attn_fwd_kernel<D, true, false>>(C::kSmemBytes))
-                          : (two ? smem_attr_once<attn_fwd_kernel<D, false, true>>(C::kSmemBytes)
-                                 : smem_attr_once<attn_fwd_kernel<D, false, false>>(C::kSmemBytes));
+    auto kernel = cross ? (two ? attn_fwd_kernel<D, true, true, kQLoad> : attn_fwd_kernel<D, true, false, kQLoad>)
+                        : (two ? attn_fwd_kernel<D, false, true, kQLoad> : attn_fwd_kernel<D, false, false, kQLoad>);
+    cudaError_t e = cross ? (two ? smem_attr_once<attn_fwd_kernel<D, true, true, kQLoad>>(smem)
+                                 : smem_attr_once<attn_fwd_kernel<D, true, false, kQLoad>>(smem))
+                          : (two ? smem_attr_once<attn_fwd_kernel<D, false, true, kQLoad>>(smem)
+                                 : smem_attr_once<attn_fwd_kernel<D, false, false, kQLoad>>(smem));
     if (e != cudaSuccess) return e;
     // Split the pairs of a last wave that would fill at most half of the SMs
     // into single-tile units (one CTA per SM).
@@ -653,9 +723,23 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     const int rem = total % nsm;
     const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;
-    const dim3 grid(q.pair_units + 2 * split);
-    kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(q.pair_units + 2 * split);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, q);
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     cudaStream_t stream) {
+    return p.q_load ? launch_dq<D, true>(p, tq, tk, tv, stream) : launch_dq<D, false>(p, tq, tk, tv, stream);
 }
 
 }  // namespace attn

@@ -65,8 +65,6 @@ __device__ __forceinline__ int tile_off(int row, int ch) {
 // 512-byte scale atom.
 __device__ __forceinline__ int atom_off(int r, int c4) { return 16 * (r & 31) + 4 * (r >> 5) + c4; }
 
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Exact 1/s for every E4M3 scale code s (0 for the zero code and NaN codes,
 // which the saturating conversion never produces).
@@ -106,19 +104,18 @@ __device__ __forceinline__ float amax16(const uint64_t (&x2)[8]) {
 }
 
 // ---------------------------------------------------------------- tiles
-// One staged 128-token tile of Q or K, quantized along d.  neg_mean: -mean
-// of K per channel (smoothing; negation is exact, so x + (-mean) is the
-// fp32 subtraction x - mean) or nullptr for Q.  Rows past N arrive as zeros
-// and get code 0 and scale 0.
-template <int D, bool kSmooth>
-__device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N, int tile,
-                                        const float *__restrict__ neg_mean, const float *__restrict__ rcp_lut,
-                                        uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, bool st32) {
-    constexpr int kBpt = D / 32;  // 16-element blocks per thread (4 or 2), consecutive along d
-    const int row = static_cast<int>(threadIdx.x) >> 1;
-    const int part = static_cast<int>(threadIdx.x) & 1;
-    const int t = tile * kTile + row;
-    uint32_t cw[2 * kBpt];
+// Quantizes the D/32 consecutive 16-element blocks of token row `row`,
+// channel half `part`, of a staged tile along d: E2M1 codes into cw (two
+// words per block), the blocks' scale codes packed one byte each into the
+// return value.  smooth: add neg_mean (-mean of K per channel; negation is
+// exact, so x + (-mean) is the fp32 subtraction x - mean) first.  The
+// attention kernel's Q-on-load path calls this too, so both produce the
+// same codes by construction.
+template <int D>
+__device__ __forceinline__ uint32_t row_part_codes(const uint8_t *__restrict__ stage, int row, int part, bool smooth,
+                                                   const float *__restrict__ neg_mean,
+                                                   const float *__restrict__ rcp_lut, uint32_t (&cw)[D / 16]) {
+    constexpr int kBpt = D / 32;
     uint32_t scw = 0;
 #pragma unroll
     for (int i = 0; i < kBpt; ++i) {
@@ -129,7 +126,7 @@ __device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N
         uint64_t x2[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) x2[e] = pack2(bf16_lo(w[e]), bf16_hi(w[e]));
-        if (kSmooth && t < N) {
+        if (smooth) {
             const float4 *nm = reinterpret_cast<const float4 *>(neg_mean + ch0);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -144,6 +141,22 @@ __device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N
         cw[2 * i + 1] = c.y;
         scw |= sc << (8 * i);
     }
+    return scw;
+}
+
+// One staged 128-token tile of Q or K, quantized along d.  neg_mean: -mean
+// of K per channel (smoothing) or nullptr for Q.  Rows past N arrive as
+// zeros and get code 0 and scale 0.
+template <int D, bool kSmooth>
+__device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N, int tile,
+                                        const float *__restrict__ neg_mean, const float *__restrict__ rcp_lut,
+                                        uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, bool st32) {
+    constexpr int kBpt = D / 32;  // 16-element blocks per thread (4 or 2), consecutive along d
+    const int row = static_cast<int>(threadIdx.x) >> 1;
+    const int part = static_cast<int>(threadIdx.x) & 1;
+    const int t = tile * kTile + row;
+    uint32_t cw[2 * kBpt];
+    const uint32_t scw = row_part_codes<D>(stage, row, part, kSmooth && t < N, neg_mean, rcp_lut, cw);
     uint8_t *dst = codes + static_cast<size_t>(t) * (D / 2) + part * (kBpt * 8);
     if constexpr (kBpt == 4) {
         if (st32) {
@@ -608,6 +621,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     quant_k_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const QuantParams p) {
     extern __shared__ uint8_t smem_raw[];
+    pdl_trigger();  // the attention launch behind this one may start its prologue
     const SmemPtrs sm = smem_setup<D>(smem_raw);
     const int ntile = p.Np / kTile;
     const long long nk = static_cast<long long>(p.BH) * ntile;

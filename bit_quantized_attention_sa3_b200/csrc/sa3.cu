@@ -102,10 +102,12 @@ int check_shape(int B, int H, int N, int d) {
     return SA3_OK;
 }
 
-int check_qkv(const sa3_qkv_fp4 *t) {
-    if (!t || !t->q_fp4 || !t->q_sf || !t->k_fp4 || !t->k_sf || !t->vt_fp4 || !t->vt_sf || !t->k_mean)
+// need_q: the Q code and scale buffers are used (not so when Q is skipped
+// by the quantizer or quantized on load by the attention kernel).
+int check_qkv(const sa3_qkv_fp4 *t, bool need_q = true) {
+    if (!t || (need_q && (!t->q_fp4 || !t->q_sf)) || !t->k_fp4 || !t->k_sf || !t->vt_fp4 || !t->vt_sf || !t->k_mean)
         return SA3_ERR_INVALID_ARG;
-    if (!aligned16(t->q_fp4) || !aligned16(t->q_sf) || !aligned16(t->k_fp4) || !aligned16(t->k_sf) ||
+    if ((need_q && (!aligned16(t->q_fp4) || !aligned16(t->q_sf))) || !aligned16(t->k_fp4) || !aligned16(t->k_sf) ||
         !aligned16(t->vt_fp4) || !aligned16(t->vt_sf) || !aligned16(t->k_mean))
         return SA3_ERR_INVALID_ARG;
     return SA3_OK;
@@ -158,18 +160,19 @@ int sa3_quantize_qkv_ex(const void *q, const void *k, const void *v, int B, int 
                         size_t workspace_bytes, struct CUstream_st *stream) {
     int rc = check_shape(B, H, Nq, d);
     if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
-    if ((flags & ~static_cast<unsigned int>(SA3_V_SMOOTH)) != 0) return SA3_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<unsigned int>(SA3_V_SMOOTH | SA3_SKIP_Q)) != 0) return SA3_ERR_INVALID_ARG;
     const bool vsmooth = (flags & SA3_V_SMOOTH) != 0;
-    if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
-    if ((rc = check_qkv(out)) != SA3_OK) return rc;
+    const bool skip_q = (flags & SA3_SKIP_Q) != 0;
+    if ((!skip_q && (!q || !aligned16(q))) || !k || !v || !aligned16(k) || !aligned16(v)) return SA3_ERR_INVALID_ARG;
+    if ((rc = check_qkv(out, !skip_q)) != SA3_OK) return rc;
     if (vsmooth && (!v_mean || !aligned16(v_mean))) return SA3_ERR_INVALID_ARG;
     const int64_t need = sa3_quant_workspace_bytes_ex(B, H, Nkv, d, flags);
     if (!workspace || !aligned16(workspace) || workspace_bytes < static_cast<size_t>(need)) return SA3_ERR_INVALID_ARG;
     {
-        const Range in[3] = {range_of(q, int64_t(B) * H * Nq * d * 2), range_of(k, int64_t(B) * H * Nkv * d * 2),
-                             range_of(v, int64_t(B) * H * Nkv * d * 2)};
-        const Range wr[9] = {range_of(out->q_fp4, sa3_qk_fp4_bytes(B, H, Nq, d)),
-                             range_of(out->q_sf, sa3_qk_sf_bytes(B, H, Nq, d)),
+        const Range in[3] = {range_of(skip_q ? nullptr : q, skip_q ? 0 : int64_t(B) * H * Nq * d * 2),
+                             range_of(k, int64_t(B) * H * Nkv * d * 2), range_of(v, int64_t(B) * H * Nkv * d * 2)};
+        const Range wr[9] = {range_of(out->q_fp4, skip_q ? 0 : sa3_qk_fp4_bytes(B, H, Nq, d)),
+                             range_of(out->q_sf, skip_q ? 0 : sa3_qk_sf_bytes(B, H, Nq, d)),
                              range_of(out->k_fp4, sa3_qk_fp4_bytes(B, H, Nkv, d)),
                              range_of(out->k_sf, sa3_qk_sf_bytes(B, H, Nkv, d)),
                              range_of(out->vt_fp4, sa3_vt_fp4_bytes(B, H, Nkv, d)),
@@ -190,17 +193,18 @@ int sa3_quantize_qkv_ex(const void *q, const void *k, const void *v, int B, int 
     p.BH = B * H;
     p.N = Nkv;
     p.Np = static_cast<int>(sa3_padded_len(Nkv));
-    p.Nq = Nq;
-    p.Npq = static_cast<int>(sa3_padded_len(Nq));
+    // skipping Q: a schedule without Q tiles
+    p.Nq = skip_q ? 0 : Nq;
+    p.Npq = skip_q ? 0 : static_cast<int>(sa3_padded_len(Nq));
     p.chunk = static_cast<int>(sa3_kmean_chunk(Nkv));
     p.nchunk = static_cast<int>(sa3_kmean_nchunk(Nkv));
-    p.st32 = aligned32(p.q_fp4) && aligned32(p.k_fp4);
+    p.st32 = (skip_q || aligned32(p.q_fp4)) && aligned32(p.k_fp4);
     p.vsmooth = vsmooth ? 1 : 0;
     p.v_mean = v_mean;
     p.vpart = p.part + static_cast<size_t>(p.BH) * p.nchunk * d;
     CUtensorMap tq, tk, tv;
-    if (!make_qkv_map(&tq, q, d, Nq, p.BH) || !make_qkv_map(&tk, k, d, Nkv, p.BH) ||
-        !make_qkv_map(&tv, v, d, Nkv, p.BH))
+    if (!make_qkv_map(&tk, k, d, Nkv, p.BH) || !make_qkv_map(&tv, v, d, Nkv, p.BH) ||
+        !(skip_q ? make_qkv_map(&tq, k, d, Nkv, p.BH) : make_qkv_map(&tq, q, d, Nq, p.BH)))
         return SA3_ERR_CUDA;
     return sa3::launch_quant(p, tq, tk, tv, d, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SA3_OK
                                                                                                         : SA3_ERR_CUDA;
@@ -280,13 +284,16 @@ int sa3_quantize_qkv_noalloc(const void *q, const void *k, const void *v, int B,
     return sa3_quantize_qkv(q, k, v, B, H, N, d, out, scratch, SA3_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean, int B, int H, int Nq, int Nkv, int d, int causal,
-                    float sm_scale, unsigned int flags, void *out, struct CUstream_st *stream) {
+int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const void *q, const float *v_mean, int B, int H, int Nq, int Nkv,
+                    int d, int causal, float sm_scale, unsigned int flags, void *out, struct CUstream_st *stream) {
     int rc = check_shape(B, H, Nq, d);
     if (rc != SA3_OK || (rc = check_shape(B, H, Nkv, d)) != SA3_OK) return rc;
-    if ((rc = check_qkv(in)) != SA3_OK) return rc;
+    if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL | SA3_V_SMOOTH | SA3_Q_ON_LOAD)) != 0)
+        return SA3_ERR_INVALID_ARG;
+    const bool q_load = (flags & SA3_Q_ON_LOAD) != 0;
+    if ((rc = check_qkv(in, !q_load)) != SA3_OK) return rc;
+    if (q_load && (!q || !aligned16(q))) return SA3_ERR_INVALID_ARG;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
-    if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL | SA3_V_SMOOTH)) != 0) return SA3_ERR_INVALID_ARG;
     if ((flags & SA3_V_SMOOTH) && (!v_mean || !aligned16(v_mean))) return SA3_ERR_INVALID_ARG;
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
@@ -295,7 +302,8 @@ int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean, int B, int H, in
     const int Np = static_cast<int>(sa3_padded_len(Nkv));
     CUtensorMap tq, tk, tv;
     const CUtensorMapSwizzle qk_sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-    if (!make_map(&tq, in->q_fp4, d / 2, static_cast<uint64_t>(BH) * Npq, d / 2, 128, qk_sw) ||
+    if (!(q_load ? make_qkv_map(&tq, q, d, Nq, BH)
+                 : make_map(&tq, in->q_fp4, d / 2, static_cast<uint64_t>(BH) * Npq, d / 2, 128, qk_sw)) ||
         !make_map(&tk, in->k_fp4, d / 2, static_cast<uint64_t>(BH) * Np, d / 2, 128, qk_sw) ||
         !make_map(&tv, in->vt_fp4, Np / 2, static_cast<uint64_t>(BH) * d, 64, d, CU_TENSOR_MAP_SWIZZLE_64B))
         return SA3_ERR_CUDA;
@@ -305,6 +313,7 @@ int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean, int B, int H, in
     p.vt_sf = static_cast<const uint8_t *>(in->vt_sf);
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.v_mean = (flags & SA3_V_SMOOTH) ? v_mean : nullptr;
+    p.q_load = q_load ? 1 : 0;
     p.BH = BH;
     p.N = Nkv;
     p.Np = Np;
@@ -321,7 +330,7 @@ int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean, int B, int H, in
 int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
                       unsigned int flags, void *out, struct CUstream_st *stream) {
     if ((flags & ~static_cast<unsigned int>(SA3_P_TWO_LEVEL)) != 0) return SA3_ERR_INVALID_ARG;
-    return sa3_attn_fwd_ex(in, nullptr, B, H, Nq, Nkv, d, causal, sm_scale, flags, out, stream);
+    return sa3_attn_fwd_ex(in, nullptr, nullptr, B, H, Nq, Nkv, d, causal, sm_scale, flags, out, stream);
 }
 
 int sa3_attn_fwd_i8_lse(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,

@@ -53,6 +53,7 @@ struct AttnParams {
     float scale_log2;  // fp32(sm_scale * log2 e)
     float p_pre_log2;  // 0, or 11 for two-level P (P scaled by 2^11 before microscaling;
                        // selects the kernel instance, whose exponent is fixed)
+    int q_load;        // FP4: 1 = Q arrives as bf16 (3-D tensor map) and is quantized in the kernel
     int npairs;        // Q-tile pairs per head (set by the launcher)
     int pair_units;    // work units that are pairs; the rest are single tiles
 };

@@ -322,4 +322,10 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFF)));
 }
 
+// Programmatic dependent launch: let the next kernel on the stream start
+// its prologue / wait until every prerequisite grid has completed and its
+// writes are visible.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace sa3

@@ -239,12 +239,26 @@ int sa3_attn_fwd_lens(const sa3_qkv_fp4 *in, int B, int H, int Nq, int Nkv, int 
  *   V smoothing needs V's mean before V can be quantized, so V is read
  *   twice (once for the sums, once to quantize).
  * SA3_P_TWO_LEVEL (attention only): as in sa3_attn_fwd_lens.
+ * SA3_SKIP_Q (quantizer) / SA3_Q_ON_LOAD (attention): Q is not quantized by
+ *   the quantizer (q, out->q_fp4 and out->q_sf may be NULL and are not
+ *   touched) and the attention kernel reads the bf16 Q itself (argument q:
+ *   bf16 [B][H][Nq][d], device, 16-byte aligned; in->q_fp4 and in->q_sf
+ *   are ignored), quantizing each 128-row tile with the same block recipe
+ *   -- bit for bit the codes and scales sa3_quantize_qkv would write --
+ *   before its first S.  This saves the quantizer's Q pass (Q's bf16 read,
+ *   its code and scale writes and their re-read) at the cost of Q's bf16
+ *   read inside the attention kernel.  The pages call the method
+ *   "plug-and-play"; this is the same computation with one HBM round trip
+ *   fewer.  Output identical to the two-pass path.
  *
- * v_mean is ignored (may be NULL) without SA3_V_SMOOTH.  Any other flag bit:
- * SA3_ERR_INVALID_ARG.  Everything else as in the _lens calls, which are
- * these with flags 0 (quantizer) or flags without SA3_V_SMOOTH (attention).
+ * v_mean is ignored (may be NULL) without SA3_V_SMOOTH, q without
+ * SA3_Q_ON_LOAD.  Any other flag bit: SA3_ERR_INVALID_ARG.  Everything else
+ * as in the _lens calls, which are these with flags 0 (quantizer) or flags
+ * of SA3_P_TWO_LEVEL only (attention).
  */
 #define SA3_V_SMOOTH 2u
+#define SA3_SKIP_Q 4u
+#define SA3_Q_ON_LOAD 8u
 static inline int64_t sa3_quant_workspace_bytes_ex(int64_t B, int64_t H, int64_t N, int64_t d, unsigned int flags)
 { return sa3_quant_workspace_bytes(B, H, N, d) * ((flags & SA3_V_SMOOTH) ? 2 : 1); }
 int sa3_quantize_qkv_ex(const void *q, const void *k, const void *v,
@@ -252,7 +266,7 @@ int sa3_quantize_qkv_ex(const void *q, const void *k, const void *v,
                         const sa3_qkv_fp4 *out, float *v_mean,
                         void *workspace, size_t workspace_bytes,
                         struct CUstream_st *stream);
-int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const float *v_mean,
+int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const void *q, const float *v_mean,
                     int B, int H, int Nq, int Nkv, int d, int causal, float sm_scale,
                     unsigned int flags, void *out, struct CUstream_st *stream);
 

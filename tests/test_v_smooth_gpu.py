@@ -104,8 +104,8 @@ def test_v_smooth_argument_checks():
                                        ctypes.byref(st), None, ws.data_ptr(), 2 * ws.numel(), stream)
     assert rc == sa3.SA3_ERR_INVALID_ARG  # no v_mean
     out = torch.empty_like(q)
-    rc = sa3.lib().sa3_attn_fwd_ex(ctypes.byref(st), None, B, H, N, N, d, 0, 0.0, sa3.SA3_V_SMOOTH, out.data_ptr(),
-                                   stream)
+    rc = sa3.lib().sa3_attn_fwd_ex(ctypes.byref(st), None, None, B, H, N, N, d, 0, 0.0, sa3.SA3_V_SMOOTH,
+                                   out.data_ptr(), stream)
     assert rc == sa3.SA3_ERR_INVALID_ARG
-    rc = sa3.lib().sa3_attn_fwd_ex(ctypes.byref(st), None, B, H, N, N, d, 0, 0.0, 4, out.data_ptr(), stream)
+    rc = sa3.lib().sa3_attn_fwd_ex(ctypes.byref(st), None, None, B, H, N, N, d, 0, 0.0, 16, out.data_ptr(), stream)
     assert rc == sa3.SA3_ERR_INVALID_ARG  # unknown flag
