@@ -99,3 +99,38 @@ def test_binding_loads_the_library_and_reports_its_version():
     for name in _declared():
         if name not in ("sa3_selftest_wait_timeout", "sa3_quantize_qkv_noalloc", "sa3_version"):
             assert getattr(L, name).argtypes, name  # ctypes leaves argtypes None unless set
+
+
+def test_binding_sizes_match_the_header(tmp_path):
+    """The binding's size helpers restate the header's inline functions:
+    compile the header's own into a host program and compare."""
+    import shutil
+
+    sa3 = pytest.importorskip("bit_quantized_attention_sa3_b200")
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("needs a C compiler")
+    shapes = [(1, 1, 1, 64), (2, 16, 4096, 128), (1, 30, 17776, 64), (4, 32, 8192, 128), (1, 256, 8192, 128),
+              (1, 32, 32768, 128), (3, 7, 1000, 64)]
+    src = tmp_path / "sizes.c"
+    lines = ['#include "sa3.h"', "#include <stdio.h>", "int main(void) {"]
+    for B, H, N, d in shapes:
+        lines.append(f'  printf("%lld %lld %lld %lld\\n", (long long)sa3_padded_len({N}), '
+                     f"(long long)sa3_kmean_chunk({N}), (long long)sa3_quant_workspace_bytes({B}, {H}, {N}, {d}), "
+                     f"(long long)sa3_quant_workspace_bytes_ex({B}, {H}, {N}, {d}, SA3_V_SMOOTH));")
+    lines.append('  printf("%u\\n", (unsigned)SA3_NOALLOC_SCRATCH_BYTES);')
+    lines.append("  return 0;\n}")
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "sizes"
+    r = subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    for (B, H, N, d), line in zip(shapes, out):
+        got = [int(x) for x in line.split()]
+        want = [sa3.padded_len(N), sa3.kmean_chunk(N), sa3.quant_workspace_bytes(B, H, N, d),
+                sa3.quant_workspace_bytes(B, H, N, d, v_smooth=True)]
+        assert got == want, (B, H, N, d)
+    # the no-alloc scratch holds exactly 256 heads of 8192 tokens at d = 128
+    assert int(out[len(shapes)]) == sa3.quant_workspace_bytes(1, 256, 8192, 128)
