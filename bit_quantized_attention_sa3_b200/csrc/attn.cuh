@@ -158,7 +158,7 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Quantizes one staged bf16 Q tile in shared memory (this thread: token row
-// t/2, channel half t%2 of the tile's 256 threads) into the layout the MMA
+// qk_row(t), channel half qk_part(t) of the tile's 256 threads) into the layout the MMA
 // reads: E2M1 codes in 64-byte (D = 128) or 32-byte (D = 64) swizzled
 // K-major rows, scales in 512-byte atoms.  The blocks are quantized by the
 // quantizer's own routine; rows past Nq arrive as zeros and get code 0,
@@ -166,8 +166,8 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 template <int D>
 __device__ __forceinline__ void quantize_q_tile(const uint8_t *__restrict__ stage, const float *__restrict__ rcp_lut,
                                                 uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, int t) {
-    const int row = t >> 1;
-    const int part = t & 1;
+    const int row = quant::qk_row(t);
+    const int part = quant::qk_part(t);
     uint32_t cw[D / 16];
     const uint32_t scw = quant::row_part_codes<D>(stage, row, part, false, nullptr, rcp_lut, cw);
     if constexpr (D == 128) {

@@ -22,7 +22,8 @@
 //      quantizes its contiguous range of tiles.
 // Thread layouts (256 threads per CTA), all conflict-free on the swizzled
 // tiles: Q/K tiles -- a thread owns D/32 consecutive 16-element blocks of
-// one token row; V tiles (quantized transposed, 16 tokens per block) -- a
+// one token row, the 8 threads of each shared-memory phase on 8 different
+// rows; V tiles (quantized transposed, 16 tokens per block) -- a
 // thread owns a pair of channels over D/64 consecutive 16-token blocks,
 // warps reading 32 consecutive channel pairs of one token row at a time;
 // K sums -- a thread owns 8 channels of every 16th (D=128) or 32nd (D=64)
@@ -75,11 +76,32 @@ __device__ __forceinline__ void fill_rcp_lut(float *lut) {
     }
 }
 
+// Token row and channel half of thread t (0..255) in a Q/K tile: eight
+// consecutive threads take one channel half of eight consecutive rows, so
+// their 16-byte shared-memory reads fall in eight different bank groups.
+__host__ __device__ __forceinline__ int qk_row(int t) { return (t & 7) | ((t >> 4) << 3); }
+__host__ __device__ __forceinline__ int qk_part(int t) { return (t >> 3) & 1; }
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// fp32(x / 6) without a division, after Brisebarre, Muller and Raina,
+// "Accelerating Correctly Rounded Floating-Point Division when the Divisor
+// Is Known in Advance" (IEEE Trans. Computers 53(8), 2004): with
+// zh = RN(1/6) and zl = RN(1/6 - zh), RN(zh*x + RN(zl*x)) is the correctly
+// rounded quotient for every fp32 x >= 2^-122.  Below that, zl*x
+// underflows and the result may be off, but it and x / 6 both lie far
+// under 2^-10, half the smallest E4M3 step, so the scale code is 0 either
+// way; x = inf is clamped to the largest float, whose quotient saturates
+// the scale just as inf / 6 does.  tests/div6_check.c checks all of this
+// for every non-negative fp32 x.
+__host__ __device__ __forceinline__ float div6(float x) {
+    x = fminf(x, 0x1.fffffep127f);
+    return fmaf(x, 0x1.555556p-3f, x * -0x1.555556p-28f);
+}
+
 // Scale code of a block: E4M3_RN_sat(fp32(amax / 6)).
-__device__ __forceinline__ uint32_t scale_code(float amax) { return cvt_e4m3(__fdiv_rn(amax, 6.0f)); }
+__device__ __forceinline__ uint32_t scale_code(float amax) { return cvt_e4m3(div6(amax)); }
 
 // E2M1 codes of 16 values times r (fp32 products, rounded once each).
 __device__ __forceinline__ uint2 codes16(const uint64_t (&x2)[8], float r) {
@@ -96,11 +118,18 @@ __device__ __forceinline__ uint2 codes16(const uint64_t (&x2)[8], float r) {
                       cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]));
 }
 
+// max(0, |x_0|, ..., |x_15|), NaNs ignored, as a tree (max is exact, so
+// any order gives the same value).
 __device__ __forceinline__ float amax16(const uint64_t (&x2)[8]) {
-    float a = 0.0f;
+    float m[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fmaxf(fabsf(lo2(x2[i])), fabsf(hi2(x2[i]))));
-    return a;
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(lo2(x2[i])), fabsf(hi2(x2[i])));
+#pragma unroll
+    for (int w = 4; w > 0; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+    }
+    return fmaxf(m[0], 0.0f);
 }
 
 // ---------------------------------------------------------------- tiles
@@ -152,8 +181,8 @@ __device__ __forceinline__ void qk_tile(const uint8_t *__restrict__ stage, int N
                                         const float *__restrict__ neg_mean, const float *__restrict__ rcp_lut,
                                         uint8_t *__restrict__ codes, uint8_t *__restrict__ sf, bool st32) {
     constexpr int kBpt = D / 32;  // 16-element blocks per thread (4 or 2), consecutive along d
-    const int row = static_cast<int>(threadIdx.x) >> 1;
-    const int part = static_cast<int>(threadIdx.x) & 1;
+    const int row = qk_row(static_cast<int>(threadIdx.x));
+    const int part = qk_part(static_cast<int>(threadIdx.x));
     const int t = tile * kTile + row;
     uint32_t cw[2 * kBpt];
     const uint32_t scw = row_part_codes<D>(stage, row, part, kSmooth && t < N, neg_mean, rcp_lut, cw);
@@ -248,15 +277,15 @@ __device__ __forceinline__ void v_tile(const uint8_t *__restrict__ stage, int N,
 // One staged 128-token tile of Q or K as INT8 with one scale for the whole
 // tile ("SageAttention" summary, "Approach"; per-block scales):
 // s = fp32(amax / 127), r = fp32(1 / s), code = clamp(rn_even(fp32(x r)),
-// +-127).  Thread: token row t/2, channel half t%2.  red: 8 floats of
+// +-127).  Thread: token row qk_row(t), channel half qk_part(t).  red: 8 floats of
 // shared scratch.  Returns nothing; thread 0 stores the scale.
 template <int D, bool kSmooth>
 __device__ __forceinline__ void qk_tile_i8(const uint8_t *__restrict__ stage, int N, int tile,
                                            const float *__restrict__ neg_mean, int8_t *__restrict__ codes,
                                            float *__restrict__ scale_out, float *red, bool st32) {
     constexpr int kCh = D / 2;  // channels per thread
-    const int row = static_cast<int>(threadIdx.x) >> 1;
-    const int part = static_cast<int>(threadIdx.x) & 1;
+    const int row = qk_row(static_cast<int>(threadIdx.x));
+    const int part = qk_part(static_cast<int>(threadIdx.x));
     const int t = tile * kTile + row;
     float x[kCh];
     float amax = 0.0f;

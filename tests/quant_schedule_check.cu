@@ -6,13 +6,27 @@
 // once to a column sum, every summed tile belongs to the chunk it is
 // reported in, every chunk is flushed exactly once (its last tile), no job
 // is out of range, and no CTA receives more than the average plus one chunk
-// of tiles.  Only host code runs.
+// of tiles; the thread -> (row, channel half) map of a Q/K tile is one to
+// one.  Only host code runs.
 #include "quant.cuh"
 
 #include <cstdio>
 #include <vector>
 
 int main() {
+    {
+        // the thread -> (row, channel half) map of a Q/K tile: one to one,
+        // and the 8 threads of each shared-memory phase on 8 row classes
+        std::vector<int> seen(256, 0);
+        for (int t = 0; t < 256; ++t) {
+            const int r = sa3::quant::qk_row(t), h = sa3::quant::qk_part(t);
+            if (r < 0 || r >= 128 || h < 0 || h > 1 || seen[2 * r + h]++ ||
+                h != sa3::quant::qk_part(t & ~7) || (r & 7) != (t & 7)) {
+                printf("qk_row / qk_part: bad map at thread %d\n", t);
+                return 1;
+            }
+        }
+    }
     long long checked = 0;
     for (int BH : {1, 2, 3, 7, 30, 32, 128, 151})
         for (int N : {1, 100, 128, 129, 300, 1000, 4096, 8192, 17776, 32768})
