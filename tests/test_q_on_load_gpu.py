@@ -111,3 +111,20 @@ def test_q_on_load_argument_checks():
     assert rc == sa3.SA3_ERR_INVALID_ARG  # Q on load without q
     rc = sa3.lib().sa3_attn_fwd_ex(ctypes.byref(st), None, None, B, H, N, N, d, 0, 0.0, 0, out.data_ptr(), stream)
     assert rc == sa3.SA3_ERR_INVALID_ARG  # no Q codes and no flag
+
+
+@pytest.mark.gpu
+def test_q_written_by_the_kernel_just_before():
+    """The attention kernel is a programmatic dependent launch: with Q on
+    load, its Q reads must still come after the preceding kernel's writes.
+    Here the kernel just before the attention launch writes the Q it reads."""
+    q, k, v = [t.cuda() for t in _qkv("noncausal_b2h16n4096d128", 1000, 1000, {"B": 1, "H": 4})]
+    kv = sa3.quantize_qkv(q, k, v, skip_q=True)
+    ref = sa3.attn_fwd(kv, q=q)
+    for i in range(3):
+        q2 = torch.empty_like(q)
+        q2.copy_(q)  # a copy kernel, enqueued right before the attention launch
+        got = sa3.attn_fwd(kv, q=q2)
+        torch.cuda.synchronize()
+        assert sa3.device_status() == sa3.SA3_OK
+        assert torch.equal(got, ref), i
