@@ -44,7 +44,7 @@ constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 16;               // 2 tiles x 2 column halves x 4 lane quadrants
 constexpr int kWarpProducer = kSoftmaxWarps;     // warp 16
 constexpr int kWarpMma = kSoftmaxWarps + 1;      // warp 17
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;  // 576 threads (at most 112 registers each)
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;  // 576 threads: the register file allows 112 each; 96 are used
 
 constexpr int kBarCountBytes = (18 + 2 * kStages) * 8;  // barrier slots below
 
@@ -157,10 +157,10 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
-// Quantizes one staged bf16 Q tile in shared memory (this thread: token row
-// qk_row(t), channel half qk_part(t) of the tile's 256 threads) into the layout the MMA
-// reads: E2M1 codes in 64-byte (D = 128) or 32-byte (D = 64) swizzled
-// K-major rows, scales in 512-byte atoms.  The blocks are quantized by the
+// Quantizes one staged bf16 Q tile in shared memory (this thread: token
+// row qk_row(t), channel half qk_part(t) of the tile's 256 threads) into
+// the layout the MMA reads: E2M1 codes in 64-byte (D = 128) or 32-byte
+// (D = 64) swizzled K-major rows, scales in 512-byte atoms.  The blocks are quantized by the
 // quantizer's own routine; rows past Nq arrive as zeros and get code 0,
 // scale 0.
 template <int D>

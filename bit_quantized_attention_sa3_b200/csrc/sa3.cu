@@ -82,9 +82,10 @@ Range range_of(const void *p, int64_t n) {
 }
 bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
 
-// True if any written range overlaps any input range.  The quantizer's
-// second launch loads K before it waits for the first launch, so an output
-// that aliases an input would race with those loads.
+// True if any written range overlaps any input range.  Every launch here
+// has CTAs reading inputs while others write outputs (the quantizer's
+// second launch also loads K before it waits for the first), so an output
+// that aliases an input would race with those reads.
 bool any_overlap(const Range *in, int nin, const Range *out, int nout) {
     for (int i = 0; i < nin; ++i)
         for (int o = 0; o < nout; ++o)
@@ -295,6 +296,21 @@ int sa3_attn_fwd_ex(const sa3_qkv_fp4 *in, const void *q, const float *v_mean, i
     if (q_load && (!q || !aligned16(q))) return SA3_ERR_INVALID_ARG;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
     if ((flags & SA3_V_SMOOTH) && (!v_mean || !aligned16(v_mean))) return SA3_ERR_INVALID_ARG;
+    {
+        // the output must not share bytes with any input: other CTAs may
+        // still be reading an input (Q on load above all) while one writes
+        const Range wr[1] = {range_of(out, int64_t(B) * H * Nq * d * 2)};
+        const Range rd[8] = {range_of(q_load ? nullptr : in->q_fp4, q_load ? 0 : sa3_qk_fp4_bytes(B, H, Nq, d)),
+                             range_of(q_load ? nullptr : in->q_sf, q_load ? 0 : sa3_qk_sf_bytes(B, H, Nq, d)),
+                             range_of(in->k_fp4, sa3_qk_fp4_bytes(B, H, Nkv, d)),
+                             range_of(in->k_sf, sa3_qk_sf_bytes(B, H, Nkv, d)),
+                             range_of(in->vt_fp4, sa3_vt_fp4_bytes(B, H, Nkv, d)),
+                             range_of(in->vt_sf, sa3_vt_sf_bytes(B, H, Nkv, d)),
+                             range_of(q_load ? q : nullptr, q_load ? int64_t(B) * H * Nq * d * 2 : 0),
+                             range_of((flags & SA3_V_SMOOTH) ? v_mean : nullptr,
+                                      (flags & SA3_V_SMOOTH) ? sa3_kmean_bytes(B, H, d) : 0)};
+        if (any_overlap(rd, 8, wr, 1)) return SA3_ERR_INVALID_ARG;
+    }
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
     const int BH = B * H;
@@ -342,6 +358,17 @@ int sa3_attn_fwd_i8_lse(const sa3_qkv_i8 *in, int B, int H, int Nq, int Nkv, int
         return SA3_ERR_INVALID_ARG;
     if (!out || !aligned16(out) || (causal != 0 && causal != 1)) return SA3_ERR_INVALID_ARG;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SA3_ERR_INVALID_ARG;
+    {
+        // no output may share bytes with an input or with the other output
+        const Range wr[2] = {range_of(out, int64_t(B) * H * Nq * d * 2),
+                             range_of(lse, lse ? int64_t(B) * H * Nq * 4 : 0)};
+        const Range rd[5] = {range_of(in->q_i8, sa3_i8_bytes(B, H, Nq, d)),
+                             range_of(in->q_scale, sa3_i8_scale_bytes(B, H, Nq)),
+                             range_of(in->k_i8, sa3_i8_bytes(B, H, Nkv, d)),
+                             range_of(in->k_scale, sa3_i8_scale_bytes(B, H, Nkv)),
+                             range_of(in->vt_f16, sa3_vt_f16_bytes(B, H, Nkv, d))};
+        if (any_overlap(rd, 5, wr, 2) || overlap(wr[0], wr[1])) return SA3_ERR_INVALID_ARG;
+    }
     if (!(sm_scale > 0.0f)) sm_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     if (!std::isfinite(sm_scale)) return SA3_ERR_INVALID_ARG;
     const int BH = B * H;

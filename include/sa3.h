@@ -35,9 +35,11 @@
  *     calls only enqueue kernels, with no allocation, synchronization or
  *     attribute call, so they can be recorded into a CUDA graph (stream
  *     capture) and replayed with new inputs in the same buffers;
- *   - the quantizer's inputs (q, k, v) must not share bytes with any of its
- *     outputs or its workspace: its second kernel starts loading K while
- *     the first may still be writing.  Such a call is rejected.
+ *   - no call's outputs may share bytes with its inputs (or its
+ *     workspace): some CTAs still read inputs while others write, and the
+ *     quantizer's second kernel starts loading K while the first may still
+ *     be writing.  Such a call is rejected, including an in-place
+ *     attention call whose output aliases the Q it quantizes on load.
  *
  * Error behaviour: arguments are checked before any launch; a bad argument
  * returns SA3_ERR_INVALID_ARG (null pointer, misalignment, non-positive

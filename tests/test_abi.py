@@ -87,6 +87,42 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.sa3_attn_fwd_lens(None, 1, 1, 8, at, 128, 0, 0.0, 0, None, None) == 2
 
 
+def test_outputs_that_alias_inputs_are_rejected_without_a_gpu(lib):
+    """The aliasing checks run on addresses alone, before any launch: an
+    attention output overlapping the Q it quantizes on load, or one of the
+    quantized operands, and an 8-bit output overlapping its log-sum-exp."""
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.sa3_attn_fwd_ex.restype = I
+    lib.sa3_attn_fwd_ex.argtypes = [P, P, P, I, I, I, I, I, I, F, ctypes.c_uint, P, P]
+    lib.sa3_attn_fwd_i8_lse.restype = I
+    lib.sa3_attn_fwd_i8_lse.argtypes = [P, I, I, I, I, I, I, F, P, P, P]
+    B, H, N, d = 1, 2, 256, 64
+    mb = 1 << 20
+    # seven buffers 1 MiB apart (fake, 16-byte aligned addresses; never touched)
+    bufs = [(i + 1) * mb for i in range(7)]
+
+    class QKV(ctypes.Structure):
+        _fields_ = [(n, ctypes.c_void_p) for n in ("q_fp4", "q_sf", "k_fp4", "k_sf", "vt_fp4", "vt_sf", "k_mean")]
+
+    st = QKV(*bufs)
+    q = 16 * mb
+    q_on_load = 8
+    # in place: out = q
+    assert lib.sa3_attn_fwd_ex(ctypes.byref(st), q, None, B, H, N, N, d, 0, 0.0, q_on_load, q, None) == 1
+    # out reaching into q's last bytes
+    assert lib.sa3_attn_fwd_ex(ctypes.byref(st), q, None, B, H, N, N, d, 0, 0.0, q_on_load, q - 16, None) == 1
+    # out over the K codes (two-pass path)
+    assert lib.sa3_attn_fwd_ex(ctypes.byref(st), None, None, B, H, N, N, d, 0, 0.0, 0, bufs[2] + 64, None) == 1
+
+    class QKV8(ctypes.Structure):
+        _fields_ = [(n, ctypes.c_void_p) for n in ("q_i8", "q_scale", "k_i8", "k_scale", "vt_f16", "k_mean")]
+
+    st8 = QKV8(*bufs[:6])
+    out = 16 * mb
+    assert lib.sa3_attn_fwd_i8_lse(ctypes.byref(st8), B, H, N, N, d, 0, 0.0, out, out + 64, None) == 1
+    assert lib.sa3_attn_fwd_i8_lse(ctypes.byref(st8), B, H, N, N, d, 0, 0.0, bufs[4], None, None) == 1
+
+
 def test_binding_loads_the_library_and_reports_its_version():
     """The Python binding's own loader (no GPU needed to load or to ask the
     version) sets every declared signature."""
