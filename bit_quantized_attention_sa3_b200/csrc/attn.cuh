@@ -721,7 +721,8 @@ cudaError_t launch_dq(const AttnParams &p, const CUtensorMap &tq, const CUtensor
     const int total = q.npairs * p.BH;
     const int nsm = sm_count();
     const int rem = total % nsm;
-    const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
+    // (all of them when even that fits in one wave: fewer rows per CTA, lower latency)
+    const int split = 2 * total <= nsm ? total : (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(q.pair_units + 2 * split);

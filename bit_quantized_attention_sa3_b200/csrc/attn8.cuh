@@ -482,7 +482,8 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     const int total = q.npairs * p.BH;
     const int nsm = sm_count();
     const int rem = total % nsm;
-    const int split = (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
+    // (all of them when even that fits in one wave: fewer rows per CTA, lower latency)
+    const int split = 2 * total <= nsm ? total : (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;
     kernel<<<dim3(q.pair_units + 2 * split), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
     return cudaGetLastError();
