@@ -221,8 +221,10 @@ def fp4_peak_probe(sa3, dev, iters=16384):
 def accuracy_sample(w, q, k, v, out, causal, two=False, vsm=False, nunits=6):
     """The output's accuracy on a seeded sample of (head, Q block) units: the
     oracle quantizes those heads itself and attends on its own operands
-    (worst per-block rel-L2 of the GPU output against it), and the fp64
-    exact attention of the bf16 inputs gives the cosines of both."""
+    (worst per-block rel-L2 of the GPU output against it, as is and with
+    bf16 rounding ties forgiven: a one-ulp bf16 difference where the
+    oracle's fp32 value lies within 2^-16 of the two values' midpoint), and
+    the fp64 exact attention of the bf16 inputs gives the cosines of both."""
     import numpy as np
     import oracle
     Nq, N = q.shape[2], k.shape[2]
@@ -239,11 +241,20 @@ def accuracy_sample(w, q, k, v, out, causal, two=False, vsm=False, nunits=6):
         return t.reshape(B * H, n, d)[heads].reshape(1, len(heads), n, d).contiguous()
     qs, ks, vs = hd(q), hd(k), hd(v)
     rq = oracle.quantize_qkv(qs, ks, vs, smooth_v=vsm)
-    ref = oracle.bf16_bits_to_f32(oracle.attn_fwd(rq, Nq, causal, units=sub, p_two_level=two))[0]
+    ref32 = np.zeros((1, len(heads), Nq, w.d), np.float32)
+    ref = oracle.bf16_bits_to_f32(oracle.attn_fwd(rq, Nq, causal, units=sub, p_two_level=two, out32=ref32))[0]
+    ref32 = ref32[0]
     ex = oracle.attn_exact(qs, ks, vs, causal, units=sub)[0]
     got = out.float().cpu().numpy().reshape(w.B * w.H, Nq, w.d)[heads]
     live = (np.arange(Nq) + (N - Nq) >= 0) if causal else np.ones(Nq, bool)
-    worst, gs, rs, es = 0.0, [], [], []
+    def tied(g, r, r32):
+        # adjacent bf16 values of one sign whose fp32 source sits on their midpoint
+        gb = (np.ascontiguousarray(g, np.float32).view(np.uint32) >> 16).astype(np.int64)
+        rb = (np.ascontiguousarray(r, np.float32).view(np.uint32) >> 16).astype(np.int64)
+        mid = (g.astype(np.float64) + r.astype(np.float64)) / 2
+        return (np.abs(gb - rb) == 1) & ((gb >> 15) == (rb >> 15)) & \
+            (np.abs(r32.astype(np.float64) - mid) <= 2.0 ** -16 * np.abs(mid))
+    worst, worst_t, gs, rs, es = 0.0, 0.0, [], [], []
     for h, qb in sub:
         rows = np.arange(qb * 128, min(Nq, qb * 128 + 128))
         rows = rows[live[rows]]
@@ -251,6 +262,8 @@ def accuracy_sample(w, q, k, v, out, causal, two=False, vsm=False, nunits=6):
             continue
         g, r, e = (a[h, rows].astype(np.float64) for a in (got, ref, ex))
         worst = max(worst, float(np.linalg.norm(g - r) / np.linalg.norm(r)))
+        gt = np.where(tied(got[h, rows], ref[h, rows], ref32[h, rows]), r, g)
+        worst_t = max(worst_t, float(np.linalg.norm(gt - r) / np.linalg.norm(r)))
         gs.append(g.ravel())
         rs.append(r.ravel())
         es.append(e.ravel())
@@ -258,7 +271,9 @@ def accuracy_sample(w, q, k, v, out, causal, two=False, vsm=False, nunits=6):
 
     def cos(a, b):
         return float(a @ b / np.sqrt((a @ a) * (b @ b)))
-    return {"rel_l2_vs_oracle_worst_block": float(f"{worst:.3e}"), "cosine_vs_exact": round(cos(g, e), 5),
+    return {"rel_l2_vs_oracle_worst_block": float(f"{worst:.3e}"),
+            "rel_l2_vs_oracle_worst_block_ties_forgiven": float(f"{worst_t:.3e}"),
+            "cosine_vs_exact": round(cos(g, e), 5),
             "oracle_cosine_vs_exact": round(cos(r, e), 5),
             "sample": f"{len(units)} (head, 128-row Q block) units; the oracle quantizes those heads itself"}
 
