@@ -188,6 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Launched as a programmatic dependent: everything above overlaps the
+    // tail of the kernel before (the quantizer); every global read below
+    // comes after it has completed
+    pdl_wait();
     const uint32_t tmem = *tmem_slot;
 
     if (warp >= kWarpProducer) {
@@ -306,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l = 0.0f;
         bool ok = true;
         for (int j = 0; j < n_i; ++j) {
+            const float skj = sk[j];  // issued before the wait for S, which hides its latency
             if (!warp_wait(bars + kBarSFull + i, j & 1, abort_flag)) {
                 ok = false;
                 break;
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float rmax = fmaxf(xs[r], xs[kBlk + r]);
             // t = S * f with f = fp32(fp32(s_q s_k) c) > 0 (floored at the
             // smallest normal so that a zero block gives t = +-0, not 0 * inf)
-            const float f = fmaxf(__fmul_rn(__fmul_rn(sq, sk[j]), c2), 1.17549435e-38f);
+            const float f = fmaxf(__fmul_rn(__fmul_rn(sq, skj), c2), 1.17549435e-38f);
             const float tmax = rmax == -INFINITY ? -INFINITY : __fmul_rn(rmax, f);
             const float m_new = kCross ? fmaxf(fmaxf(m, tmax), -3.402823466e38f) : fmaxf(m, tmax);
             const float nm = -m_new;
@@ -485,8 +490,17 @@ cudaError_t launch_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorM
     // (all of them when even that fits in one wave: fewer rows per CTA, lower latency)
     const int split = 2 * total <= nsm ? total : (total > nsm && rem > 0 && 2 * rem <= nsm) ? rem : 0;
     q.pair_units = total - split;
-    kernel<<<dim3(q.pair_units + 2 * split), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, q);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(q.pair_units + 2 * split);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, q);
 }
 
 }  // namespace attn8
