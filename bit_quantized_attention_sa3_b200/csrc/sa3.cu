@@ -14,6 +14,12 @@
 #include <cuda_runtime.h>
 
 #include "sa3.h"
+
+// Only the C entry points of sa3.h are exported.  The kernels, their host
+// stubs and launchers stay hidden, so that a second build of this library
+// (or any library with the same template instances) loaded into the process
+// can neither bind to them nor interpose its own.
+#pragma GCC visibility push(hidden)
 #include "sa3_internal.h"
 #include "sm100.cuh"
 
@@ -21,6 +27,7 @@
 #include "attn8.cuh"
 #include "probe.cuh"
 #include "quant.cuh"
+#pragma GCC visibility pop
 
 namespace {
 

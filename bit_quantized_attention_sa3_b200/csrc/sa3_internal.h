@@ -58,6 +58,13 @@ struct AttnParams {
     int pair_units;    // work units that are pairs; the rest are single tiles
 };
 
+// The two host helpers below keep per-process caches in function-local
+// statics.  They have internal linkage: as inline functions of namespace
+// scope the compiler would export those statics as process-wide unique
+// symbols, and two builds of this library loaded into one process would then
+// share them (the second build would skip raising its own kernels' limit).
+namespace {
+
 // Host: raise Kernel's dynamic shared memory limit once per device (the
 // attribute persists in the device's module), so that later calls -- those
 // recorded into a CUDA graph included -- make no attribute call.  Devices
@@ -90,5 +97,7 @@ inline int sm_count() {
     if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
+
+}  // namespace
 
 }  // namespace sa3

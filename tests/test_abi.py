@@ -4,6 +4,8 @@ before touching the device."""
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -35,6 +37,18 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in _declared():
         assert hasattr(lib, name), name
+
+
+@pytest.mark.skipif(shutil.which("nm") is None, reason="needs binutils nm")
+def test_library_exports_only_the_declared_symbols(lib):
+    """The kernels, their launchers and the host helpers' caches stay inside
+    the library: a second build loaded into the same process (or another
+    library with the same template instances) must not bind to them."""
+    from bit_quantized_attention_sa3_b200 import build
+    r = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True, check=True)
+    syms = [ln.split() for ln in r.stdout.splitlines() if len(ln.split()) == 3]
+    assert sorted(name for _, kind, name in syms if kind in "TtWwVvuBDR") == _declared()
+    assert not [name for _, kind, name in syms if kind == "u"], "process-wide unique symbols"
 
 
 def test_version(lib):
