@@ -16,7 +16,11 @@
 //              is shared by two threads that exchange partial row maxima
 //   warps 8-15 softmax for Q tile 1
 //   warp 16    producer: TMA loads of Q, and of K / V^T codes + scales into
-//              a 3-stage ring (mbarrier transaction counts)
+//              a 6-stage ring (mbarrier transaction counts).  A slot stays
+//              held from S = Q K^T until O += P V of both tiles, about two
+//              blocks, so the ring runs four blocks ahead of the MMAs; at
+//              d = 128 six stages were 1.5-2 % faster than three, and seven
+//              or eight no faster (the Q-on-load instance has room for six)
 //   warp 17    allocates TMEM and issues every tcgen05 op from one thread:
 //              scale-factor copies (tcgen05.cp), S = Q K^T, O += P V
 // TMEM (512 columns): S (128, shared by both tiles -- each softmax group
@@ -40,7 +44,7 @@ namespace sa3 {
 namespace attn {
 
 constexpr int kBlk = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 6;
 constexpr int kSoftmaxWarps = 16;               // 2 tiles x 2 column halves x 4 lane quadrants
 constexpr int kWarpProducer = kSoftmaxWarps;     // warp 16
 constexpr int kWarpMma = kSoftmaxWarps + 1;      // warp 17
