@@ -48,7 +48,11 @@ constexpr int kStages = 6;
 constexpr int kSoftmaxWarps = 16;               // 2 tiles x 2 column halves x 4 lane quadrants
 constexpr int kWarpProducer = kSoftmaxWarps;     // warp 16
 constexpr int kWarpMma = kSoftmaxWarps + 1;      // warp 17
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;  // 576 threads: the register file allows 112 each; 96 are used
+// 576 threads.  Warps are placed on the SM's four sub-partitions in turn, so
+// two of them hold 5 warps; a sub-partition's 16384 registers then allow 96
+// per thread (allocation granularity 8), which is what the launch bound
+// gives the compiler, and what the kernel uses
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 
 constexpr int kBarCountBytes = (18 + 2 * kStages) * 8;  // barrier slots below
 
