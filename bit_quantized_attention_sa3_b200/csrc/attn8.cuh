@@ -19,7 +19,8 @@
 // scale columns in TMEM); S is int32 and becomes fp32 exactly through the
 // 1.5 * 2^23 bias trick (|S| <= 127 * 127 * 128 < 2^22); P is 16 bits, so a
 // P tile is two 64-key 128-byte-swizzled atoms (32 KB) and a V^T tile two
-// 64-key atoms of d rows; two KV stages at d = 128 (three at d = 64).
+// 64-key atoms of d rows; K and V^T have rings of their own (three K and
+// two V^T slots at d = 128, four and three at d = 64).
 #pragma once
 
 #include "attn.cuh"
@@ -40,7 +41,14 @@ using attn::warp_wait;
 template <int D>
 struct Cfg {
     static constexpr int al(int x) { return (x + 1023) & ~1023; }
-    static constexpr int kStages = D == 128 ? 2 : 3;
+    // K and V^T in rings of their own: a K slot is free once both tiles'
+    // S = Q K^T have run, a V^T slot only after both O += P V, so K can be
+    // fetched further ahead than a shared K + V^T slot would allow
+    static constexpr int kKStages = D == 128 ? 3 : 4;
+    static constexpr int kVStages = D == 128 ? 2 : 3;
+    // the producer issues K(j + kLead) before V^T(j): then both wait for
+    // slots that the same MMA iteration frees
+    static constexpr int kLead = kKStages + 1 - kVStages;
     static constexpr int kQBytes = kBlk * D;               // int8 Q or K tile: 128 rows x D bytes
     static constexpr int kAtomBytes = kBlk * 128;          // 128 rows x 64 halves
     static constexpr int kVAtomBytes = D * 128;            // D rows x 64 halves
@@ -51,11 +59,11 @@ struct Cfg {
     // shared memory map, offsets from a 1024-byte aligned base
     static constexpr int oQ0 = 0;
     static constexpr int oQ1 = al(oQ0 + kQBytes);
-    static constexpr int oStage = al(oQ1 + kQBytes);
-    static constexpr int sK = 0;
-    static constexpr int sV = al(kQBytes);
-    static constexpr int kStageBytes = al(sV + kVBytes);
-    static constexpr int oP0 = oStage + kStages * kStageBytes;
+    static constexpr int oK = al(oQ1 + kQBytes);          // K ring
+    static constexpr int kKSlot = al(kQBytes);
+    static constexpr int oV = oK + kKStages * kKSlot;     // V^T ring
+    static constexpr int kVSlot = al(kVBytes);
+    static constexpr int oP0 = oV + kVStages * kVSlot;
     static constexpr int oP1 = oP0 + kPBytes;
     static constexpr int oXch = oP1 + kPBytes;             // row maxima [2 parity][2 tiles][2 halves][128]
     static constexpr int oXl = oXch + 4096;                // row sums [2 tiles][2 halves][128]
@@ -69,19 +77,24 @@ struct Cfg {
     static constexpr uint32_t kTmemCols = 512;
 };
 
-constexpr int kMaxStages = 3;
+constexpr int kMaxK = 4, kMaxV = 3;
 enum : int {
     kBarQ = 0,
-    kBarKvFull = 1,                    // kMaxStages
-    kBarKvEmpty = 1 + kMaxStages,      // kMaxStages
-    kBarSFull = 1 + 2 * kMaxStages,    // 2
-    kBarSEmpty = 3 + 2 * kMaxStages,   // 1
-    kBarPFull = 4 + 2 * kMaxStages,    // 2
-    kBarPvDone = 6 + 2 * kMaxStages,   // 2
-    kBarDrain = 8 + 2 * kMaxStages,    // 1
-    kBarXch = 9 + 2 * kMaxStages,      // 8
-    kBarCount = 17 + 2 * kMaxStages
+    kBarKFull = 1,                                  // kMaxK
+    kBarKEmpty = kBarKFull + kMaxK,                 // kMaxK
+    kBarVFull = kBarKEmpty + kMaxK,                 // kMaxV
+    kBarVEmpty = kBarVFull + kMaxV,                 // kMaxV
+    kBarSFull = kBarVEmpty + kMaxV,                 // 2
+    kBarSEmpty = kBarSFull + 2,                     // 1
+    kBarPFull = kBarSEmpty + 1,                     // 2
+    kBarPvDone = kBarPFull + 2,                     // 2
+    kBarDrain = kBarPvDone + 2,                     // 1
+    kBarXch = kBarDrain + 1,                        // 8
+    kBarCount = kBarXch + 8
 };
+static_assert(Cfg<128>::kKStages <= kMaxK && Cfg<64>::kKStages <= kMaxK && Cfg<128>::kVStages <= kMaxV &&
+                  Cfg<64>::kVStages <= kMaxV,
+              "ring barriers");
 static_assert(kBarCount * 8 + 8 <= 256, "barrier area");
 
 // Instruction descriptors (dense, K-major A and B, M = 128):
@@ -128,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn8_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
     using C = Cfg<D>;
-    constexpr int kStages = C::kStages;
+    constexpr int kK = C::kKStages;
+    constexpr int kV = C::kVStages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -165,9 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bars + kBarQ, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(bars + kBarKvFull + s, 1);
-            mbar_init(bars + kBarKvEmpty + s, 1);
+        for (int s = 0; s < kK; ++s) {
+            mbar_init(bars + kBarKFull + s, 1);
+            mbar_init(bars + kBarKEmpty + s, 1);
+        }
+        for (int s = 0; s < kV; ++s) {
+            mbar_init(bars + kBarVFull + s, 1);
+            mbar_init(bars + kBarVEmpty + s, 1);
         }
         mbar_init(bars + kBarSFull + 0, 1);
         mbar_init(bars + kBarSFull + 1, 1);
@@ -205,23 +223,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bq, (valid1 ? 2u : 1u) * C::kQBytes);
             tma_load_2d(base + C::oQ0, &tm_q, 0, bh * p.Npq + tile0 * kBlk, bq);
             if (valid1) tma_load_2d(base + C::oQ1, &tm_q, 0, bh * p.Npq + tile1 * kBlk, bq);
-            int issued = 0;
-            for (int j = 0; j < nmax; ++j) {
-                const int s = j % kStages;
-                const int r = j / kStages;
-                if (r > 0 && !mbar_wait(bars + kBarKvEmpty + s, (r - 1) & 1, abort_flag)) break;
-                uint8_t *st = base + C::oStage + s * C::kStageBytes;
-                uint64_t *bf = bars + kBarKvFull + s;
-                mbar_arrive_expect_tx(bf, C::kQBytes + C::kVBytes);
-                tma_load_2d(st + C::sK, &tm_k, 0, bh * p.Np + j * kBlk, bf);
-                // V^T: keys 64a .. 64a+63 of block j for every channel, two 128-byte-wide boxes
-                tma_load_2d(st + C::sV, &tm_v, j * 256, bh * D, bf);
-                tma_load_2d(st + C::sV + C::kVAtomBytes, &tm_v, j * 256 + 128, bh * D, bf);
-                issued = j + 1;
+            // step t: K(t), then V^T(t - kLead); a wait for a slot depends
+            // only on MMA iterations that the loads issued before it feed
+            int k_issued = 0, v_issued = 0;
+            for (int t = 0; t < nmax + C::kLead; ++t) {
+                if (t < nmax) {
+                    const int s = t % kK;
+                    const int r = t / kK;
+                    if (r > 0 && !mbar_wait(bars + kBarKEmpty + s, (r - 1) & 1, abort_flag)) break;
+                    uint64_t *bf = bars + kBarKFull + s;
+                    mbar_arrive_expect_tx(bf, C::kQBytes);
+                    tma_load_2d(base + C::oK + s * C::kKSlot, &tm_k, 0, bh * p.Np + t * kBlk, bf);
+                    k_issued = t + 1;
+                }
+                const int j = t - C::kLead;
+                if (j >= 0 && j < nmax) {
+                    const int s = j % kV;
+                    const int r = j / kV;
+                    if (r > 0 && !mbar_wait(bars + kBarVEmpty + s, (r - 1) & 1, abort_flag)) break;
+                    uint8_t *sv = base + C::oV + s * C::kVSlot;
+                    uint64_t *bf = bars + kBarVFull + s;
+                    mbar_arrive_expect_tx(bf, C::kVBytes);
+                    // V^T: keys 64a .. 64a+63 of block j for every channel, two 128-byte-wide boxes
+                    tma_load_2d(sv, &tm_v, j * 256, bh * D, bf);
+                    tma_load_2d(sv + C::kVAtomBytes, &tm_v, j * 256 + 128, bh * D, bf);
+                    v_issued = j + 1;
+                }
             }
             drain_wait(bq, 0);
-            for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
-                drain_wait(bars + kBarKvFull + j % kStages, (j / kStages) & 1);
+            for (int j = k_issued - kK < 0 ? 0 : k_issued - kK; j < k_issued; ++j)
+                drain_wait(bars + kBarKFull + j % kK, (j / kK) & 1);
+            for (int j = v_issued - kV < 0 ? 0 : v_issued - kV; j < v_issued; ++j)
+                drain_wait(bars + kBarVFull + j % kV, (j / kV) & 1);
         }
     } else {
         // ----------------------------------------------------------- MMA
@@ -229,14 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdQK = idesc_i8(128);
             constexpr uint32_t kIdPV = idesc_f16(D);
             int nqk = 0;
-            auto stage_s = [&](int j) -> uint32_t {
-                return base_s + C::oStage + static_cast<uint32_t>(j % kStages) * C::kStageBytes;
-            };
             auto issue_qk = [&](int i, int j) -> bool {
                 if (nqk > 0 && !mbar_wait(bars + kBarSEmpty, (nqk - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t qa = base_s + (i ? C::oQ1 : C::oQ0);
-                const uint32_t kb = stage_s(j) + C::sK;
+                const uint32_t kb = base_s + C::oK + static_cast<uint32_t>(j % kK) * C::kKSlot;
 #pragma unroll
                 for (int kc = 0; kc < D / 32; ++kc)  // K = 32 int8 per instruction
                     tc_mma_i8(tmem + C::tS, sdesc_kmajor_sw(qa + 32 * kc, C::kQKSbo, C::kQKLayout),
@@ -249,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(bars + kBarPFull + i, j & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t pa = base_s + (i ? C::oP1 : C::oP0);
-                const uint32_t vb = stage_s(j) + C::sV;
+                const uint32_t vb = base_s + C::oV + static_cast<uint32_t>(j % kV) * C::kVSlot;
 #pragma unroll
                 for (int kc = 0; kc < 8; ++kc) {  // K = 16 halves per instruction, 4 per 64-key atom
                     const uint32_t a = pa + (kc >> 2) * C::kAtomBytes + 32 * (kc & 3);
@@ -262,23 +292,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
 
             bool ok = mbar_wait(bars + kBarQ, 0, abort_flag);
-            if (ok && nmax > 0) ok = mbar_wait(bars + kBarKvFull + 0, 0, abort_flag);
+            if (ok && nmax > 0) ok = mbar_wait(bars + kBarKFull + 0, 0, abort_flag);
             if (ok && nmax > 0) {
                 tc_fence_after();
                 if (n0 > 0) ok = issue_qk(0, 0);
                 if (ok && n1 > 0) ok = issue_qk(1, 0);
+                if (ok) tc_commit(bars + kBarKEmpty + 0);
             }
             for (int j = 0; ok && j < nmax; ++j) {
                 if (j + 1 < nmax) {
-                    ok = mbar_wait(bars + kBarKvFull + (j + 1) % kStages, ((j + 1) / kStages) & 1, abort_flag);
+                    ok = mbar_wait(bars + kBarKFull + (j + 1) % kK, ((j + 1) / kK) & 1, abort_flag);
                     if (!ok) break;
-                    tc_fence_after();
                 }
+                ok = mbar_wait(bars + kBarVFull + j % kV, (j / kV) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
                 if (j + 1 < n0 && !(ok = issue_qk(0, j + 1))) break;
                 if (j < n0 && !(ok = issue_pv(0, j))) break;
                 if (j + 1 < n1 && !(ok = issue_qk(1, j + 1))) break;
+                // K(j + 1) has been read by both S products
+                if (j + 1 < nmax) tc_commit(bars + kBarKEmpty + (j + 1) % kK);
                 if (j < n1 && !(ok = issue_pv(1, j))) break;
-                tc_commit(bars + kBarKvEmpty + j % kStages);
+                tc_commit(bars + kBarVEmpty + j % kV);
             }
             tc_commit(bars + kBarDrain);
             drain_wait(bars + kBarDrain, 0);
