@@ -52,6 +52,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP = 3              # sa3_quantize_qkv: 2 kernels; sa3_attn_fwd: 1
+EX2_PER_SM_CLK = 16                # ex2.approx.ftz.f32 results per SM per clock (measured on a B200)
+EX2_PER_S = 1.0 + 1.0 / 16 + 1.0 / 64  # FP4 attention: P, one block scale per 16 keys, alpha per row half
 
 
 def parse():
@@ -291,6 +293,26 @@ def attn_ops(w, Nq):
     return 4.0 * w.B * w.H * pairs * w.d
 
 
+def processed_s_elements(B, H, Nq, N, causal):
+    """S elements the attention kernels compute: whole 128 x 128 tiles, for
+    each Q tile the KV blocks up to the one holding its last row's diagonal
+    (causal; the last query lines up with the last key), all of them else."""
+    nqt, nkvt, off = (Nq + 127) // 128, (N + 127) // 128, N - Nq
+    total = 0
+    for t in range(nqt):
+        last = t * 128 + 127 + off
+        total += min(last // 128 + 1, nkvt) if (causal and last >= 0) else (0 if causal else nkvt)
+    return B * H * total * 128 * 128
+
+
+def exp2_ceiling_us(B, H, Nq, N, causal, sm_mhz, n_sm):
+    """Time the FP4 attention kernel would take if its exp2 unit were busy
+    every cycle: EX2_PER_S exponentials per computed S element at
+    EX2_PER_SM_CLK per SM per clock, at the sampled SM clock."""
+    n = processed_s_elements(B, H, Nq, N, causal) * EX2_PER_S
+    return n / (EX2_PER_SM_CLK * n_sm * sm_mhz * 1e6) * 1e6
+
+
 def make_inputs(w, Nq, seed):
     """The workload's seeded q, k, v; q cut to (or drawn with) Nq tokens."""
     if Nq <= w.N:
@@ -511,6 +533,16 @@ def run_sa3(args, rank, world, local):
         line["roofline"]["peak_bf16x4"] = round(peak_rule, 1)
         line["roofline"]["frac_of_bf16x4"] = round(achieved / peak_rule, 4)
         line["roofline"]["peak_bf16x4_source"] = f"{src} bf16 burst {pk['bf16_tflops']} x 4 (nominal FP4/bf16 ratio)"
+        try:  # the kernel's binding limit: its exponentials (never fails the line)
+            mhz = line["clocks"].get("sm_mhz") or line["clocks"].get("sm_max_mhz")
+            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            ceil_us = exp2_ceiling_us(B, H, Nq, N, causal, float(mhz), n_sm)
+            line["roofline"]["exp2_ceiling"] = {
+                "us": round(ceil_us, 1), "frac": round(ceil_us / (t_attn * 1e3), 4),
+                "how": (f"{EX2_PER_S:.4f} ex2 per computed S element (whole 128x128 tiles) at "
+                        f"{EX2_PER_SM_CLK} per SM per clock, {n_sm} SMs, {mhz} MHz")}
+        except Exception as e:  # noqa: BLE001
+            line["roofline"]["exp2_ceiling"] = {"us": None, "error": repr(e)[:120]}
     if Nq != N:
         line["config"]["Nq"] = Nq
         line["config"]["ops"] = "4*d per (query, key) pair the mask leaves"

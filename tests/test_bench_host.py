@@ -99,3 +99,31 @@ def test_gpu_arm_prints_the_contract_line():
     assert line["gpu_launches"] == 3 * line["steps"]
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(line["clocks"])
     assert line["e2e"]["h2d_bytes_per_step"] == 3 * 2 * 16 * 4096 * 128 * 2
+
+
+def _tiles_brute(Nq, N, causal):
+    """Q tile t computes KV block b when some row of t sees some key of b."""
+    n = 0
+    for t in range((Nq + 127) // 128):
+        for b in range((N + 127) // 128):
+            if not causal:
+                n += 1
+                continue
+            last_row = t * 128 + 127            # rows past Nq still belong to the tile
+            if b * 128 <= last_row + (N - Nq):  # the block's first key is visible to the last row
+                n += 1
+    return n
+
+
+@pytest.mark.parametrize("Nq,N,causal", [(4096, 4096, False), (256, 256, True), (300, 300, True), (77, 1000, True),
+                                         (1000, 130, True), (1, 300, True), (17776, 17776, False),
+                                         (8192, 8192, True), (130, 1000, False)])
+def test_processed_s_elements_counts_the_kernels_tiles(bench, Nq, N, causal):
+    assert bench.processed_s_elements(2, 3, Nq, N, causal) == 2 * 3 * _tiles_brute(Nq, N, causal) * 128 * 128
+
+
+def test_exp2_ceiling_of_the_headline_shape(bench):
+    # 2*16*4096^2 S elements x (1 + 1/16 + 1/64) exp2 / (16 per SM-clock x 148 SMs x 1.965 GHz)
+    us = bench.exp2_ceiling_us(2, 16, 4096, 4096, False, 1965.0, 148)
+    assert abs(us - 2 * 16 * 4096 * 4096 * 1.078125 / (16 * 148 * 1965e6) * 1e6) < 1e-6
+    assert 124.0 < us < 125.0
