@@ -22,7 +22,9 @@ lands writes its block into its slot, an MMA checks when the pipe executes
 it that its K / V^T slots, P buffer and S buffer hold what it means to read
 or overwrite, and a softmax group checks that S holds its own product.
 It covers tiles with no key (causal, more queries than keys), tile 1 longer
-than tile 0, one KV block, and more blocks than slots.
+than tile 0, one KV block, and more blocks than slots.  The same machinery
+checks the two halves of a row exchanging partial row maxima through slots
+double-buffered by block parity, and their row sums at the end.
 """
 import random
 
@@ -34,8 +36,10 @@ class Deadlock(Exception):
 
 
 class Sim:
-    def __init__(self, rng):
+    def __init__(self, rng, arrivals=None):
         self.rng = rng
+        self.need = dict(arrivals or {})  # barrier -> arrivals per phase (default 1)
+        self.arrived = {}
         self.count = {}          # barrier -> completed phases
         self.waiting = {}        # agent -> (barrier, phase index it waits for)
         self.pending_loads = []  # (barrier, slot, block) of TMA loads in flight
@@ -121,7 +125,11 @@ class Sim:
                 elif req[0] == "commit":
                     self.pipe.append(("commit", req[1]))
                 elif req[0] == "arrive":
-                    self.complete(req[1])
+                    bar = req[1]
+                    self.arrived[bar] = self.arrived.get(bar, 0) + 1
+                    if self.arrived[bar] == self.need.get(bar, 1):
+                        self.arrived[bar] = 0
+                        self.complete(bar)
                 step(name)
 
 
@@ -350,5 +358,56 @@ def test_the_model_catches_a_broken_protocol():
             Sim(random.Random(seed)).run(i8_agents(8, 8, 3, 2, early_k_release=True))
         except AssertionError as e:
             assert "reads" in str(e), e
+            caught += 1
+    assert caught > 0
+
+
+def exchange_agents(n_i):
+    """The two halves of a row in one tile (attn.cuh and attn8.cuh softmax):
+    per KV block each writes its partial row maximum into the slot of the
+    block's parity, arrives on the pair's barrier (both halves per phase)
+    and reads the other half's value; after the last block the row sums go
+    through a slot of their own and the same barrier's next phase."""
+    def half(h):
+        def agent():
+            for j in range(n_i):
+                yield ("write", ("xch", j & 1, h), j)
+                yield ("arrive", "xbar")
+                yield wait("xbar", j)
+                yield ("check", ("xch", j & 1, 1 - h), j)
+            if n_i > 0:
+                yield ("write", ("xl", h), "sum")
+                yield ("arrive", "xbar")
+                yield wait("xbar", n_i)
+                yield ("check", ("xl", 1 - h), "sum")
+        return agent
+    return {"half0": half(0), "half1": half(1)}
+
+
+@pytest.mark.parametrize("n_i", [1, 2, 3, 8, 33])
+def test_row_max_exchange_double_buffer(n_i):
+    for seed in range(200):
+        Sim(random.Random(seed), arrivals={"xbar": 2}).run(exchange_agents(n_i))
+
+
+def test_row_max_exchange_needs_both_slots():
+    """Planted mistake: one slot for every block.  A fast half then
+    overwrites the value its partner has not read yet."""
+    def one_slot(n_i):
+        def half(h):
+            def agent():
+                for j in range(n_i):
+                    yield ("write", ("xch", 0, h), j)
+                    yield ("arrive", "xbar")
+                    yield wait("xbar", j)
+                    yield ("check", ("xch", 0, 1 - h), j)
+            return agent
+        return {"half0": half(0), "half1": half(1)}
+
+    caught = 0
+    for seed in range(200):
+        try:
+            Sim(random.Random(seed), arrivals={"xbar": 2}).run(one_slot(8))
+        except AssertionError:
             caught += 1
     assert caught > 0
