@@ -1,6 +1,7 @@
 """Host-side logic of bench.py that needs no GPU: the operation count for
 unequal query / key lengths (4*d per (query, key) pair the mask leaves,
-checked against a brute-force count of the mask) and the input shapes."""
+checked against a brute-force count of the mask), the input shapes, and
+the tiles behind the exp2 ceiling (against a brute-force tile count)."""
 import dataclasses
 import importlib.util
 import os
