@@ -37,16 +37,20 @@ BLK = 128
 VEC = 16
 
 
+def gcc_command(src: str, out: str) -> list[str]:
+    """The compiler command for the oracle: no fast math, no FMA contraction."""
+    return ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+            "-fno-fast-math", "-ffp-contract=off", "-Wall", "-Wextra",
+            "-Wno-unused-parameter", src, "-o", out, "-lm"]
+
+
 def build(force: bool = False) -> str:
     """Compile sa3_oracle.c into liboracle.so next to it (gcc + OpenMP)."""
     if (not force and os.path.exists(_LIB_PATH)
             and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
         return _LIB_PATH
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-fno-fast-math", "-ffp-contract=off", "-Wall", "-Wextra",
-           "-Wno-unused-parameter", _SRC, "-o", tmp, "-lm"]
-    subprocess.run(cmd, check=True)
+    subprocess.run(gcc_command(_SRC, tmp), check=True)
     os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -56,7 +60,10 @@ def _load():
     with _lock:
         if _lib is not None:
             return _lib
-        lib = ctypes.CDLL(build())
+        # SA3_ORACLE_LIB: a library built elsewhere from a copy of the source
+        # (the pin suite's own mutation test runs the pins against copies
+        # with a planted mistake); unset, the in-tree build
+        lib = ctypes.CDLL(os.environ.get("SA3_ORACLE_LIB") or build())
         P = ctypes.c_void_p
         I = ctypes.c_int
         F = ctypes.c_float
