@@ -24,7 +24,8 @@ or overwrite, and a softmax group checks that S holds its own product.
 It covers tiles with no key (causal, more queries than keys), tile 1 longer
 than tile 0, one KV block, and more blocks than slots.  The same machinery
 checks the two halves of a row exchanging partial row maxima through slots
-double-buffered by block parity, and their row sums at the end.
+double-buffered by block parity, and their row sums at the end, and the
+Q-on-load start (the softmax groups quantize Q before the first S product).
 """
 import random
 
@@ -137,10 +138,18 @@ def wait(bar, c):
     return ("wait", bar, c)
 
 
-def softmax(i, n_i):
+def softmax(i, n_i, q_on_load=False, valid=True):
     """One Q tile's softmax group: S in, S buffer released, P out once the
-    previous P V is done, the last P V awaited before the epilogue."""
+    previous P V is done, the last P V awaited before the epilogue.  With Q
+    on load it first waits for the bf16 Q tiles, quantizes its own (when its
+    tile exists) into the MMA's Q buffer and arrives on the Q-ready barrier
+    (both groups arrive, whether or not tile 1 exists)."""
     def agent():
+        if q_on_load:
+            yield wait("Q", 0)
+            if valid:
+                yield ("write", ("Qcodes", i), "q")
+            yield ("arrive", "QReady")
         for j in range(n_i):
             yield wait(("SFull", i), j)
             yield ("check", "S", (i, j))
@@ -154,11 +163,15 @@ def softmax(i, n_i):
     return agent
 
 
-def mma_common(n0, n1, k_ready, v_ready, after_qk, after_pv, k_slot, v_slot, early_k_release=False):
+def mma_common(n0, n1, k_ready, v_ready, after_qk, after_pv, k_slot, v_slot, early_k_release=False,
+               q_on_load=False, q_barrier=None):
     """The MMA thread's schedule, shared by both kernels: S products of both
     tiles for block 0, then per block j: S0(j+1), PV0(j), S1(j+1), PV1(j).
     k_slot(j) / v_slot(j): the buffers holding K and V^T of block j.
-    early_k_release plants a mistake: K(j+1) released before S1(j+1)."""
+    early_k_release plants a mistake: K(j+1) released before S1(j+1).
+    q_on_load: the S products read the Q codes the softmax groups wrote;
+    q_barrier: the barrier waited for before the first S product (default:
+    Q-ready with Q on load, the Q load else)."""
     nmax = max(n0, n1)
     nqk = [0]
     last_s = [None]  # the S product the next one overwrites (read by then)
@@ -166,7 +179,8 @@ def mma_common(n0, n1, k_ready, v_ready, after_qk, after_pv, k_slot, v_slot, ear
     def issue_qk(i, j):
         if nqk[0] > 0:
             yield wait("SEmpty", nqk[0] - 1)
-        yield ("mma", ((k_slot(j), j), ("S", last_s[0])), (("S", (i, j)),))
+        q_read = ((("Qcodes", i), "q"),) if q_on_load else ()
+        yield ("mma", ((k_slot(j), j), ("S", last_s[0])) + q_read, (("S", (i, j)),))
         last_s[0] = (i, j)
         yield ("commit", ("SFull", i))
         nqk[0] += 1
@@ -177,7 +191,7 @@ def mma_common(n0, n1, k_ready, v_ready, after_qk, after_pv, k_slot, v_slot, ear
         yield ("commit", ("PvDone", i))
 
     def agent():
-        yield wait("Q", 0)
+        yield wait(q_barrier or ("QReady" if q_on_load else "Q"), 0)
         if nmax == 0:
             return
         yield from k_ready(0)
@@ -206,8 +220,11 @@ def mma_common(n0, n1, k_ready, v_ready, after_qk, after_pv, k_slot, v_slot, ear
     return agent
 
 
-def fp4_agents(n0, n1, stages):
-    """attn.cuh: one ring of K, its scales, V^T and its scales per block."""
+def fp4_agents(n0, n1, stages, q_on_load=False, mma_waits_q_ready=True):
+    """attn.cuh: one ring of K, its scales, V^T and its scales per block.
+    q_on_load: the softmax groups quantize the bf16 Q tiles the producer
+    loads; mma_waits_q_ready=False plants a mistake (the MMA waits only for
+    the bf16 load)."""
     nmax = max(n0, n1)
 
     def producer():
@@ -234,8 +251,10 @@ def fp4_agents(n0, n1, stages):
     def slot(j):
         return ("KV", j % stages)
 
-    return {"producer": producer, "mma": mma_common(n0, n1, k_ready, nothing, nothing, after_pv, slot, slot),
-            "softmax0": softmax(0, n0), "softmax1": softmax(1, n1)}
+    mma = mma_common(n0, n1, k_ready, nothing, nothing, after_pv, slot, slot, q_on_load=q_on_load,
+                     q_barrier=None if mma_waits_q_ready else "Q")
+    return {"producer": producer, "mma": mma,
+            "softmax0": softmax(0, n0, q_on_load, True), "softmax1": softmax(1, n1, q_on_load, n1 > 0)}
 
 
 def i8_agents(n0, n1, k_stages, v_stages, early_k_release=False):
@@ -408,6 +427,23 @@ def test_row_max_exchange_needs_both_slots():
     for seed in range(200):
         try:
             Sim(random.Random(seed), arrivals={"xbar": 2}).run(one_slot(8))
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+@pytest.mark.parametrize("n0,n1", [(1, 0), (3, 3), (6, 7), (13, 13), (0, 1)])
+def test_fp4_q_on_load_hand_off(n0, n1):
+    for seed in range(60):
+        Sim(random.Random(seed), arrivals={"QReady": 2}).run(fp4_agents(n0, n1, 6, q_on_load=True))
+
+
+def test_q_on_load_without_the_ready_barrier_is_caught():
+    caught = 0
+    for seed in range(200):
+        try:
+            Sim(random.Random(seed), arrivals={"QReady": 2}).run(
+                fp4_agents(6, 7, 6, q_on_load=True, mma_waits_q_ready=False))
         except AssertionError:
             caught += 1
     assert caught > 0
